@@ -1,0 +1,204 @@
+"""CPU oracle for the W8A8 linear hot path -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its binding) never imports, links or calls it, and it shares no code with
+that path: the arithmetic lives in ``zq_oracle.c`` (plain C loops, compiled
+with ``gcc -O2 -ffp-contract=off``), and this module only marshals numpy
+arrays and composes the C steps in the order the sources give.
+
+Sources (web pages):
+  [ZQ]   "[2022 NeurIPS] ZeroQuant: Efficient and Affordable Post-Training
+         Quantization for Large-Scale Transformers" -- token-wise and
+         group-wise quantization paragraphs; fused-kernel flowcharts.
+  [TS36] "探秘Transformer系列之（36）— 大模型量化方案" -- §1.1.2, §1.2.2.
+  [IQ]   "Integer Quantization: Deep Dive" -- quantization formula,
+         fake quantization, quantization error.
+
+Every function here is pinned by ``tests/test_oracle_pins.py`` against
+hand-worked examples (``tests/golden/``), closed forms, invariants and
+library routines; none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "zq_oracle.c")
+_LIB = os.path.join(_HERE, "_build", "libzqoracle.so")
+
+ACT_NONE = 0
+ACT_GELU = 1
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle to ``oracle/_build/libzqoracle.so`` (no GPU)."""
+    os.makedirs(os.path.dirname(_LIB), exist_ok=True)
+    stale = (not os.path.exists(_LIB)) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC)
+    if force or stale:
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+               "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _L():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P, I64, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float
+        sig = {
+            "zqo_quantize_span": [P, I64, P, P],
+            "zqo_quantize_weights": [P, I64, I64, I64, P, P],
+            "zqo_quantize_rows": [P, I64, I64, P, P],
+            "zqo_layernorm": [P, I64, I64, P, P, F, P],
+            "zqo_bias_act": [P, I64, I64, P, ctypes.c_int, P],
+            "zqo_gemm_i32": [P, I64, I64, P, I64, P],
+            "zqo_dequant": [P, I64, I64, P, P, I64, P, ctypes.c_int, P],
+        }
+        for name, args in sig.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def _c(a, dtype):
+    a = np.ascontiguousarray(a, dtype=dtype)
+    return a, a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _chk(rc, what):
+    if rc == 2:
+        raise OracleError(f"{what}: int32 accumulator overflow")
+    if rc != 0:
+        raise OracleError(f"{what}: bad argument (status {rc})")
+
+
+def quantize_span(v):
+    """Absmax symmetric quantization of one vector ([TS36] §1.1.2).
+    Returns (int8 codes, fp32 scale)."""
+    v, pv = _c(v, np.float32)
+    q = np.empty(v.shape, np.int8)
+    s = np.zeros(1, np.float32)
+    _chk(_L().zqo_quantize_span(pv, v.size, q.ctypes.data, s.ctypes.data), "quantize_span")
+    return q, s[0]
+
+
+def quantize_weights(W, group_rows):
+    """Group-wise weight quantization ([ZQ]; [TS36] §1.2.2): W fp32 [N, K]
+    -> (Wq int8 [N, K], s_grp fp32 [N / group_rows])."""
+    W, pw = _c(W, np.float32)
+    N, K = W.shape
+    Wq = np.empty((N, K), np.int8)
+    s = np.empty(N // group_rows if group_rows > 0 else 0, np.float32)
+    _chk(_L().zqo_quantize_weights(pw, N, K, group_rows, Wq.ctypes.data, s.ctypes.data),
+         "quantize_weights")
+    return Wq, s
+
+
+def quantize_rows(Y):
+    """Per-token (row) quantization of fp32 Y [T, H] -> (q int8, s_tok fp32 [T])."""
+    Y, py = _c(Y, np.float32)
+    T, H = Y.shape
+    q = np.empty((T, H), np.int8)
+    s = np.empty(T, np.float32)
+    _chk(_L().zqo_quantize_rows(py, T, H, q.ctypes.data, s.ctypes.data), "quantize_rows")
+    return q, s
+
+
+def layernorm(x, gamma, beta, eps):
+    """LayerNorm in double, rounded to fp32 (biased variance, eps inside sqrt)."""
+    x, px = _c(x, np.float32)
+    g, pg = _c(gamma, np.float32)
+    b, pb = _c(beta, np.float32)
+    T, H = x.shape
+    y = np.empty((T, H), np.float32)
+    _chk(_L().zqo_layernorm(px, T, H, pg, pb, float(eps), y.ctypes.data), "layernorm")
+    return y
+
+
+def bias_act(x, bias=None, act=ACT_NONE):
+    """y = act(x + bias) in double, rounded to fp32 (act: identity or exact GeLU)."""
+    x, px = _c(x, np.float32)
+    T, H = x.shape
+    pb = None
+    if bias is not None:
+        bias, pb = _c(bias, np.float32)
+    y = np.empty((T, H), np.float32)
+    _chk(_L().zqo_bias_act(px, T, H, pb, int(act), y.ctypes.data), "bias_act")
+    return y
+
+
+def gemm_i32(xq, Wq):
+    """acc[t, o] = sum_k xq[t, k] * Wq[o, k], exact, int32 result."""
+    xq, px = _c(xq, np.int8)
+    Wq, pw = _c(Wq, np.int8)
+    T, K = xq.shape
+    N, K2 = Wq.shape
+    if K != K2:
+        raise OracleError("gemm_i32: K mismatch")
+    acc = np.empty((T, N), np.int32)
+    _chk(_L().zqo_gemm_i32(px, T, K, pw, N, acc.ctypes.data), "gemm_i32")
+    return acc
+
+
+def dequant(acc, s_tok, s_grp, group_rows, bias=None, act=ACT_NONE):
+    """y = act(s_tok[t] * s_grp[o // G] * acc[t, o] + bias[o]) in double -> fp32."""
+    acc, pa = _c(acc, np.int32)
+    st, ps = _c(s_tok, np.float32)
+    sg, pg = _c(s_grp, np.float32)
+    T, N = acc.shape
+    pb = None
+    if bias is not None:
+        bias, pb = _c(bias, np.float32)
+    y = np.empty((T, N), np.float32)
+    _chk(_L().zqo_dequant(pa, T, N, ps, pg, group_rows, pb, int(act), y.ctypes.data),
+         "dequant")
+    return y
+
+
+# ---- compositions, in the order of the fused flowcharts of [ZQ] ----------
+
+def ln_quant(x, gamma, beta, eps):
+    """Fused "LN + Quantize": LayerNorm, then per-token quantization."""
+    return quantize_rows(layernorm(x, gamma, beta, eps))
+
+
+def act_quant(x, bias=None, act=ACT_NONE):
+    """Fused "GeLU + Quantize" (or plain token quantization when act is none)."""
+    return quantize_rows(bias_act(x, bias, act))
+
+
+def linear(xq, s_tok, Wq, s_grp, group_rows, bias=None, act=ACT_NONE):
+    """Fused "GEMM + DeQuantize": int32 GEMM then the dequant epilogue, fp32 out."""
+    return dequant(gemm_i32(xq, Wq), s_tok, s_grp, group_rows, bias, act)
+
+
+def linear_requant(xq, s_tok, Wq, s_grp, group_rows, bias=None, act=ACT_GELU):
+    """GEMM + DeQuantize + act, then per-token quantization for the next layer."""
+    return quantize_rows(linear(xq, s_tok, Wq, s_grp, group_rows, bias, act))
+
+
+def ffn_block(x, gamma, beta, eps, W1q, s1, b1, W2q, s2, b2, group_rows):
+    """Transformer FFN as the fused kernels run it:
+    LN+quant -> GEMM1+dequant+bias+GeLU+requant -> GEMM2+dequant+bias (fp32).
+    Returns the fp32 output and the intermediate (q1, s_tok1, q2, s_tok2)."""
+    q1, st1 = ln_quant(x, gamma, beta, eps)
+    q2, st2 = linear_requant(q1, st1, W1q, s1, group_rows, b1, ACT_GELU)
+    y = linear(q2, st2, W2q, s2, group_rows, b2, ACT_NONE)
+    return y, (q1, st1, q2, st2)

@@ -1,0 +1,190 @@
+/*
+ * zq_oracle.c -- plain, slow, CPU reference of the W8A8 linear hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file; only the test suite, the smoke check and the CPU-baseline
+ * leg of the benchmark do.  It shares no code, header, table or constant
+ * with the CUDA library.
+ *
+ * Every function is the plain definition of one step, written as loops in
+ * the order the sources state it.  Floating point runs in double except
+ * where the method itself fixes fp32 (the quantizer: scale = absmax/127 and
+ * the code rint(v * (127/absmax)) are fp32 operations by definition).
+ *
+ * Sources (web pages) and the passages each function follows:
+ *   [ZQ]   "[2022 NeurIPS] ZeroQuant: Efficient and Affordable Post-Training
+ *          Quantization for Large-Scale Transformers" -- group-wise weight
+ *          quantization paragraph; token-wise activation quantization
+ *          paragraph; the fused-kernel flowcharts (LN/GeLU + Quantize,
+ *          GEMM + DeQuantize).
+ *   [TS36] "探秘Transformer系列之（36）— 大模型量化方案" -- §1.1.2
+ *          (absmax quantization to [-127,127]; vector-wise quantization,
+ *          denormalisation by the outer product of row and column scales);
+ *          §1.2.2 (dynamic per-token activation quantization fused with the
+ *          preceding LayerNorm; INT32 accumulators scaled by the weight and
+ *          activation scales before the FP16 write; group-wise weights).
+ *   [IQ]   "Integer Quantization: Deep Dive" -- "如何进行量化？" (quantize
+ *          with scale, zero-point, round-to-nearest and clamp); "量化模拟"
+ *          (dequantize x = s * (x_int - z)); "量化误差" (rounding error is
+ *          at most s/2).
+ *
+ * Readings where the pages are silent (each one is a choice, stated once):
+ *   R1 round-to-nearest ties go to even (rintf under the default mode);
+ *   R2 symmetric codes are clamped to [-127, 127], zero-point z = 0;
+ *   R3 the code is rint(v * (127/absmax)) with 127/absmax an fp32 division,
+ *      never v / scale;
+ *   R4 an all-zero vector gets scale 0 and all-zero codes;
+ *   R5 weight groups are G contiguous output rows spanning all K columns;
+ *   R6 LayerNorm uses the biased variance with eps inside the square root;
+ *   R7 GeLU is the exact erf form 0.5 x (1 + erf(x / sqrt 2));
+ *   R8 bias is added after dequantization, in floating point.
+ *
+ * Status codes: 0 = ok, 1 = bad argument, 2 = int32 overflow in the GEMM.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#define ZQO_OK 0
+#define ZQO_EARG 1
+#define ZQO_EOVERFLOW 2
+
+/* [TS36] §1.1.2 absmax rule + readings R1-R4.  One scale for the n values
+ * v[0..n): scale = absmax/127 (fp32), q_i = clamp(rint(v_i * (127/absmax))). */
+int zqo_quantize_span(const float* v, int64_t n, int8_t* q, float* scale)
+{
+    if (!v || !q || !scale || n <= 0) return ZQO_EARG;
+    float amax = 0.0f;
+    for (int64_t i = 0; i < n; ++i) {
+        float a = fabsf(v[i]);
+        if (a > amax) amax = a;
+    }
+    if (amax == 0.0f) {
+        *scale = 0.0f;
+        for (int64_t i = 0; i < n; ++i) q[i] = 0;
+        return ZQO_OK;
+    }
+    float s = amax / 127.0f;
+    float inv = 127.0f / amax;
+    for (int64_t i = 0; i < n; ++i) {
+        float t = v[i] * inv;      /* one fp32 rounding, no fused add */
+        float r = rintf(t);        /* half-to-even under FE_TONEAREST */
+        if (r > 127.0f) r = 127.0f;
+        if (r < -127.0f) r = -127.0f;
+        q[i] = (int8_t)r;
+    }
+    *scale = s;
+    return ZQO_OK;
+}
+
+/* [ZQ] group-wise weight quantization, [TS36] §1.2.2, reading R5.
+ * W is [N, K] row-major; group g holds rows g*G .. g*G+G-1 (all K columns)
+ * and is quantized as one span.  Wq is [N, K], s_grp is [N/G]. */
+int zqo_quantize_weights(const float* W, int64_t N, int64_t K, int64_t G,
+                         int8_t* Wq, float* s_grp)
+{
+    if (!W || !Wq || !s_grp || N <= 0 || K <= 0 || G <= 0 || N % G != 0)
+        return ZQO_EARG;
+    for (int64_t g = 0; g < N / G; ++g) {
+        int rc = zqo_quantize_span(W + g * G * K, G * K, Wq + g * G * K, &s_grp[g]);
+        if (rc) return rc;
+    }
+    return ZQO_OK;
+}
+
+/* Dynamic per-token quantization ([ZQ] token-wise paragraph, [TS36] §1.2.2):
+ * every row of Y [T, H] gets its own scale. */
+int zqo_quantize_rows(const float* Y, int64_t T, int64_t H, int8_t* q, float* s_tok)
+{
+    if (!Y || !q || !s_tok || T <= 0 || H <= 0) return ZQO_EARG;
+    for (int64_t t = 0; t < T; ++t) {
+        int rc = zqo_quantize_span(Y + t * H, H, q + t * H, &s_tok[t]);
+        if (rc) return rc;
+    }
+    return ZQO_OK;
+}
+
+/* LayerNorm over each row of x [T, H] in double (reading R6), result rounded
+ * once to fp32.  mean = sum/H; var = sum (x-mean)^2 / H (two passes);
+ * y = (x - mean) / sqrt(var + eps) * gamma + beta. */
+int zqo_layernorm(const float* x, int64_t T, int64_t H, const float* gamma,
+                  const float* beta, float eps, float* y)
+{
+    if (!x || !gamma || !beta || !y || T <= 0 || H <= 0) return ZQO_EARG;
+    for (int64_t t = 0; t < T; ++t) {
+        const float* r = x + t * H;
+        double mean = 0.0;
+        for (int64_t h = 0; h < H; ++h) mean += (double)r[h];
+        mean /= (double)H;
+        double var = 0.0;
+        for (int64_t h = 0; h < H; ++h) {
+            double d = (double)r[h] - mean;
+            var += d * d;
+        }
+        var /= (double)H;
+        double denom = sqrt(var + (double)eps);
+        for (int64_t h = 0; h < H; ++h) {
+            double v = ((double)r[h] - mean) / denom * (double)gamma[h] + (double)beta[h];
+            y[t * H + h] = (float)v;
+        }
+    }
+    return ZQO_OK;
+}
+
+/* Reading R7: exact GeLU in double. */
+static double gelu_d(double v) { return 0.5 * v * (1.0 + erf(v / sqrt(2.0))); }
+
+/* Element-wise activation step before token quantization ([ZQ] fused
+ * "LN/GeLU + Quantize" flowchart): y = act(x + bias), bias optional
+ * (length H, broadcast over rows), act 0 = identity, 1 = GeLU. */
+int zqo_bias_act(const float* x, int64_t T, int64_t H, const float* bias, int act, float* y)
+{
+    if (!x || !y || T <= 0 || H <= 0 || (act != 0 && act != 1)) return ZQO_EARG;
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t h = 0; h < H; ++h) {
+            double v = (double)x[t * H + h];
+            if (bias) v += (double)bias[h];
+            if (act == 1) v = gelu_d(v);
+            y[t * H + h] = (float)v;
+        }
+    return ZQO_OK;
+}
+
+/* INT8 x INT8 -> INT32 contraction ([TS36] §1.2.2 "INT32 accumulation";
+ * [IQ] MAC unit): acc[t, o] = sum_k xq[t, k] * Wq[o, k].  Accumulated in
+ * int64; a sum outside the int32 range is reported, not wrapped. */
+int zqo_gemm_i32(const int8_t* xq, int64_t T, int64_t K, const int8_t* Wq, int64_t N,
+                 int32_t* acc)
+{
+    if (!xq || !Wq || !acc || T <= 0 || K <= 0 || N <= 0) return ZQO_EARG;
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t o = 0; o < N; ++o) {
+            int64_t s = 0;
+            for (int64_t k = 0; k < K; ++k)
+                s += (int64_t)xq[t * K + k] * (int64_t)Wq[o * K + k];
+            if (s > INT32_MAX || s < INT32_MIN) return ZQO_EOVERFLOW;
+            acc[t * N + o] = (int32_t)s;
+        }
+    return ZQO_OK;
+}
+
+/* Dequantize the accumulators ([TS36] §1.2.2: scale the INT32 accumulation
+ * by the activation and weight scales; §1.1.2: denormalise by the outer
+ * product of the row and column scales; [IQ] "量化模拟" with z = 0), then add
+ * bias (reading R8) and apply the optional activation, all in double:
+ *   y[t, o] = act(s_tok[t] * s_grp[o / G] * acc[t, o] + bias[o]). */
+int zqo_dequant(const int32_t* acc, int64_t T, int64_t N, const float* s_tok,
+                const float* s_grp, int64_t G, const float* bias, int act, float* y)
+{
+    if (!acc || !s_tok || !s_grp || !y || T <= 0 || N <= 0 || G <= 0 || N % G != 0 ||
+        (act != 0 && act != 1))
+        return ZQO_EARG;
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t o = 0; o < N; ++o) {
+            double v = (double)s_tok[t] * (double)s_grp[o / G] * (double)acc[t * N + o];
+            if (bias) v += (double)bias[o];
+            if (act == 1) v = gelu_d(v);
+            y[t * N + o] = (float)v;
+        }
+    return ZQO_OK;
+}
