@@ -1,0 +1,529 @@
+"""Benchmark of the W8A8 linear hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One JSON line on stdout (rank 0).  A step is one pass of the whole inference
+path over one batch of seeded synthetic input already resident in HBM; the
+default workload is the BERT-base-shaped FFN block:
+    x bf16 [4096, 768] -> fused LayerNorm + per-token quant
+      -> W1 [3072, 768] INT8 GEMM + dequant + bias + GeLU + per-token requant
+      -> W2 [768, 3072] INT8 GEMM + dequant + bias -> bf16 [4096, 768].
+Weight group quantization is offline (done once before timing).
+
+Metric: INT8 tera-operations per second of the whole step (2*T*N*K integer
+ops per GEMM, summed, over the step time), with the fused LN/token-quant
+bandwidth and the per-kernel roofline alongside.
+
+Timing: each stage is one CUDA graph of the library's C-ABI calls; every
+timed step is preceded by a 256 MiB write that flushes the 126 MB L2 and is
+bracketed by CUDA events on the launching stream (the flush is outside the
+events).  W >= 3 warm-up steps; K timed steps; barrier + synchronize on both
+sides; the maximum over ranks.  Multi-GPU runs are independent replicas
+(the path needs no exchange): value = ops of all ranks / max time.
+
+--impl reference times the CPU oracle (the plain C reference of the same
+path) on the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from w8a8_post_quantized_b200 import inputs  # noqa: E402
+
+# Roofline denominators measured on this GPU pool (fallback if the file is absent).
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SPEC_INT8_TOPS = 4500.0          # dense INT8 tensor-core peak, spec
+SPEC_HBM_GBS = 8000.0
+INT8_OVER_BF16 = 2.0             # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return dict(FALLBACK_PEAKS, source="fallback")
+
+
+# ------------------------------------------------------------- distributed
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def reduce_max(value: float) -> float:
+    """Maximum of a per-rank scalar over all ranks (identity when single-process)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(value)
+    backend = dist.get_backend()
+    dev = torch.device("cuda", torch.cuda.current_device()) if backend == "nccl" else torch.device("cpu")
+    t = torch.tensor([float(value)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) of the GPU this rank uses."""
+
+    QUERY = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        rows = []
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 10:
+                continue
+            if self.uuid and self.uuid not in f[1]:
+                continue
+            rows.append(f)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i] == "Active"})
+        loaded = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------- workloads
+
+class Workload:
+    """A workload prepared on the device: stage callables of the public API."""
+
+    def __init__(self, name, zq, torch, device):
+        self.name = name
+        self.zq, self.torch, self.device = zq, torch, device
+        self.stages = []          # (label, fn) run in order; each one stage of the step
+        self.ops = 0              # integer ops of the GEMMs per step
+        self.tokens = 0
+        self.h2d = None           # (pinned host tensor, device tensor) of the step's input
+        self.d2h = None           # (device tensor, pinned host tensor) of the step's result
+        self.kernel_units = {}    # stage label -> (bound, algorithmic units per launch, unit)
+        self.config = {}
+
+    def dev(self, a):
+        return self.torch.from_numpy(np.ascontiguousarray(a)).to(self.device)
+
+    def dev_act(self, a):
+        if a.bf16 is not None:
+            return self.torch.from_numpy(a.bf16.view(np.int16)).to(self.device).view(self.torch.bfloat16)
+        return self.dev(a.f32)
+
+
+def build_workload(name, zq, torch, device):
+    W = Workload(name, zq, torch, device)
+    if name in ("bert_ffn", "gptj_qkv", "tiny"):
+        w = {"bert_ffn": inputs.bert_ffn, "gptj_qkv": inputs.gptj_qkv, "tiny": inputs.tiny}[name]()
+    elif name == "neox_decode":
+        w = inputs.neox_decode()
+    elif name.startswith("gemm_sweep_"):
+        M = int(name.split("_")[-1])
+        w = inputs.gemm_sweep_point(M, inputs.GEMM_SWEEP_M.index(M))
+    elif name.startswith("ln_sweep_"):
+        T, H = (int(v) for v in name.split("_")[-2:])
+        idx = inputs.LN_SWEEP_T.index(T) * len(inputs.LN_SWEEP_H) + inputs.LN_SWEEP_H.index(H)
+        w = inputs.ln_sweep_point(T, H, idx)
+    else:
+        raise SystemExit(f"unknown workload {name}")
+    x = W.dev_act(w.x)
+    T, K = x.shape
+    W.tokens = T
+    xbytes = x.numel() * x.element_size()
+    W.config = {"workload": w.name, "tokens": T, "hidden": K, "x_dtype": w.x.dtype}
+    q1 = torch.empty((T, K), dtype=torch.int8, device=device)
+    st1 = torch.empty(T, dtype=torch.float32, device=device)
+    if w.gamma is not None:
+        g, b = W.dev(w.gamma), W.dev(w.beta)
+        W.stages.append(("ln_quant", lambda: zq.zq_ln_quant(x, g, b, w.eps, q=q1, s_tok=st1)))
+        label_q = "ln_quant"
+    else:
+        W.stages.append(("act_quant", lambda: zq.zq_act_quant(x, q=q1, s_tok=st1)))
+        label_q = "act_quant"
+    # algorithmic bytes of the quantizer: read x, write codes and scales (+ gamma, beta)
+    W.kernel_units[label_q] = ("hbm", xbytes + T * K + 4 * T + (8 * K if w.gamma is not None else 0),
+                               "bytes")
+    W.h2d_src = x
+    if not w.layers:          # LN sweep point: the quantizer alone
+        W.out = q1
+        W.config.update(layers=[])
+        return W
+    layers = []
+    for lin in w.layers:
+        Wq, sg = zq.zq_quantize_weights(W.dev(lin.W), lin.group_rows)
+        layers.append((Wq, sg, W.dev(lin.bias), lin.group_rows))
+    torch.cuda.synchronize()
+    a_q, a_s = q1, st1
+    for i, (Wq, sg, b, G) in enumerate(layers):
+        N = Wq.shape[0]
+        last = i == len(layers) - 1
+        act = w.act if i == 0 else 0
+        if last:
+            out_kind = {"bf16": zq.ZQ_OUT_BF16, "f32": zq.ZQ_OUT_F32}[w.out]
+            y = torch.empty((T, N), dtype=torch.bfloat16 if w.out == "bf16" else torch.float32,
+                            device=device)
+            s_out, ws = None, None
+        else:
+            out_kind = zq.ZQ_OUT_I8_REQUANT
+            y = torch.empty((T, N), dtype=torch.int8, device=device)
+            s_out = torch.empty(T, dtype=torch.float32, device=device)
+            ws = torch.empty(zq.zq_w8a8_linear_workspace(T, Wq.shape[1], N, out_kind),
+                             dtype=torch.uint8, device=device)
+
+        def fn(a_q=a_q, a_s=a_s, Wq=Wq, sg=sg, b=b, G=G, act=act, out_kind=out_kind, y=y,
+               s_out=s_out, ws=ws):
+            zq.zq_w8a8_linear(a_q, a_s, Wq, sg, G, bias=b, act=act, out_kind=out_kind, y=y,
+                              s_tok_out=s_out, workspace=ws)
+        label = f"linear{i + 1}"
+        W.stages.append((label, fn))
+        Kd = Wq.shape[1]
+        ops = 2 * T * N * Kd
+        W.ops += ops
+        W.kernel_units[label] = ("tensor", ops, "ops")
+        a_q, a_s = y, s_out
+        W.out = y
+    W.config.update(layers=[list(l[0].shape) + [l[3]] for l in layers],
+                    epilogue=("gelu+requant" if len(layers) > 1 else ("gelu" if w.act else "bias")),
+                    out_dtype=w.out)
+    return W
+
+
+# ------------------------------------------------------------------ timing
+
+def time_device(W, steps, warmup, torch):
+    """Per-stage CUDA graphs; flush L2 before each step; CUDA events around
+    each stage on the launching stream.  Returns per-step and per-stage ms."""
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=W.device)
+    for _, fn in W.stages:       # eager warm-up (sets kernel attributes, loads modules)
+        fn()
+    torch.cuda.synchronize()
+    graphs = []
+    cap = torch.cuda.Stream()
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        for label, fn in W.stages:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                fn()
+            graphs.append((label, g))
+    stream.wait_stream(cap)
+    torch.cuda.synchronize()
+    n = len(graphs)
+
+    def run(k, record):
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(k)]
+        for s in range(k):
+            flush.zero_()
+            evs[s][0].record(stream)
+            for i, (_, g) in enumerate(graphs):
+                g.replay()
+                evs[s][i + 1].record(stream)
+        return evs
+
+    run(warmup, False)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    evs = run(steps, True)
+    torch.cuda.synchronize()
+    barrier()
+    per_step = [e[0].elapsed_time(e[-1]) for e in evs]
+    per_stage = {label: [e[i].elapsed_time(e[i + 1]) for e in evs] for i, (label, _) in enumerate(graphs)}
+    del graphs
+    return per_step, per_stage
+
+
+def time_e2e(W, steps, warmup, torch):
+    """Same step through the public API with host buffers: pinned host input
+    -> device, the stage calls, result -> pinned host, all inside the events."""
+    stream = torch.cuda.current_stream()
+    src = W.h2d_src
+    host_in = torch.empty(src.shape, dtype=src.dtype, pin_memory=True)
+    host_in.copy_(src.cpu())
+    out = W.out
+    host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=W.device)
+
+    def step():
+        src.copy_(host_in, non_blocking=True)
+        for _, fn in W.stages:
+            fn()
+        host_out.copy_(out, non_blocking=True)
+
+    for _ in range(warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(steps):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b.record(stream)
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    h2d = host_in.numel() * host_in.element_size()
+    d2h = host_out.numel() * host_out.element_size()
+    return statistics.mean(times), h2d, d2h
+
+
+def count_launches(W, zq, torch):
+    before = zq.zq_launch_count()
+    for _, fn in W.stages:
+        fn()
+    torch.cuda.synchronize()
+    return zq.zq_launch_count() - before
+
+
+# ---------------------------------------------------------- CPU baseline
+
+def oracle_sample(name, budget_s=12.0, max_rows=None):
+    """Time the CPU oracle on a bounded row sample of the workload.  Returns
+    (ops done, seconds, rows, total rows).  The oracle is single-threaded."""
+    import oracle
+    if name == "bert_ffn":
+        w = inputs.bert_ffn()
+    elif name == "gptj_qkv":
+        w = inputs.gptj_qkv()
+    elif name == "neox_decode":
+        w = inputs.neox_decode()
+    elif name == "tiny":
+        w = inputs.tiny()
+    elif name.startswith("gemm_sweep_"):
+        M = int(name.split("_")[-1])
+        w = inputs.gemm_sweep_point(M, inputs.GEMM_SWEEP_M.index(M))
+    else:
+        raise SystemExit(f"no oracle baseline for {name}")
+    qlayers = [(*oracle.quantize_weights(l.W, l.group_rows), l.bias, l.group_rows) for l in w.layers]
+    T = w.x.f32.shape[0]
+    rows_done, ops, t_total = 0, 0, 0.0
+    chunk = 8 if T >= 8 else T
+    limit = max_rows if max_rows is not None else T
+    while rows_done < limit and t_total < budget_s:
+        r0 = rows_done % T
+        x = w.x.f32[r0:r0 + chunk]
+        t0 = time.perf_counter()
+        if w.gamma is not None:
+            q, s = oracle.ln_quant(x, w.gamma, w.beta, w.eps)
+        else:
+            q, s = oracle.quantize_rows(x)
+        for i, (Wq, sg, b, G) in enumerate(qlayers):
+            act = w.act if i == 0 else 0
+            if i < len(qlayers) - 1:
+                q, s = oracle.linear_requant(q, s, Wq, sg, G, b, act)
+            else:
+                oracle.linear(q, s, Wq, sg, G, b, act)
+            ops += 2 * x.shape[0] * Wq.shape[0] * Wq.shape[1]
+        t_total += time.perf_counter() - t0
+        rows_done += x.shape[0]
+    return ops, t_total, rows_done, T
+
+
+# -------------------------------------------------------------------- main
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="bert_ffn")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args(argv)
+    if a.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    rank, world, local_rank = dist_env()
+
+    if a.impl == "reference":
+        return main_reference(a, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+    from w8a8_post_quantized_b200 import zq
+    zq.lib()
+
+    W = build_workload(a.workload, zq, torch, device)
+    launches_per_step = count_launches(W, zq, torch)
+    zq.zq_device_status()
+
+    props = torch.cuda.get_device_properties(device)
+    clocks = ClockSampler(str(getattr(props, "uuid", "")) or None)
+    clocks.start()
+    per_step, per_stage = time_device(W, a.steps, a.warmup, torch)
+    clk = clocks.stop()
+    zq.zq_device_status()
+    local_ms = sum(per_step)
+    max_ms = reduce_max(local_ms)
+    ms_per_step = max_ms / a.steps
+
+    e2e_ms, h2d, d2h = time_e2e(W, max(3, min(a.steps, 20)), 3, torch)
+    e2e_ms = reduce_max(e2e_ms)
+    zq.zq_device_status()
+
+    peaks = load_peaks()
+    int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+    stage_ms = {k: statistics.mean(v) for k, v in per_stage.items()}
+    # dominant kernel: the stage that is a single launch of the tcgen05 GEMM
+    # with the largest time (a quantizer when the workload has no GEMM)
+    gemm_stages = [k for k in stage_ms if k.startswith("linear")]
+    single = [k for k in gemm_stages if W.config.get("epilogue") != "gelu+requant" or k != "linear1"]
+    dom = max(single or gemm_stages or list(stage_ms), key=lambda k: stage_ms[k])
+    bound, units, kind = W.kernel_units[dom]
+    if bound == "tensor":
+        achieved = units / (stage_ms[dom] * 1e-3) / 1e12
+        roof = {"kernel": f"w8a8_gemm ({dom})", "bound": "tensor", "achieved": round(achieved, 1),
+                "peak": round(int8_peak, 1), "unit": "TOPS", "frac": round(achieved / int8_peak, 4),
+                "peak_source": f"{peaks['source']} bf16 burst x {INT8_OVER_BF16:g} (nominal int8/bf16)",
+                "frac_vs_spec": round(achieved / SPEC_INT8_TOPS, 4), "traffic": None}
+    else:
+        achieved = units / (stage_ms[dom] * 1e-3) / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "peak_source": f"{peaks['source']} copy bandwidth",
+                "frac_vs_spec": round(achieved / SPEC_HBM_GBS, 4), "traffic": None}
+    qlabel = "ln_quant" if "ln_quant" in stage_ms else "act_quant"
+    qb = W.kernel_units[qlabel][1]
+    q_gbs = qb / (stage_ms[qlabel] * 1e-3) / 1e9
+
+    if W.ops:
+        metric, unit = "W8A8 linear INT8 TOPS (whole step, incl. fused LN/token-quant)", "TOPS"
+        value = world * W.ops / (ms_per_step * 1e-3) / 1e12
+        e2e_value = world * W.ops / (e2e_ms * 1e-3) / 1e12
+    else:
+        metric, unit = "fused LN/token-quant GB/s", "GB/s"
+        value = world * qb / (ms_per_step * 1e-3) / 1e9
+        e2e_value = world * qb / (e2e_ms * 1e-3) / 1e9
+
+    out = {
+        "metric": metric, "value": round(value, 2), "unit": unit, "n_gpus": world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic (seeded; layer shapes only, random weights)",
+        "config": dict(W.config, parallelism=f"replicas x{world}",
+                       l2="flushed (256 MiB write) before every timed step",
+                       timing="per-stage CUDA graphs, CUDA events on the launching stream"),
+        "tokens_per_s": round(world * W.tokens / (ms_per_step * 1e-3), 1),
+        "stages_ms": {k: round(v, 5) for k, v in stage_ms.items()},
+        "ln_quant_gbs": round(q_gbs, 1),
+        "ln_quant_frac_hbm": round(q_gbs / peaks["hbm_gbs"], 4),
+        "roofline": roof,
+        "e2e": {"value": round(e2e_value, 3), "unit": unit, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": launches_per_step * a.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not a.no_cpu_baseline and W.ops:
+        ops, secs, rows, T = oracle_sample(a.workload, budget_s=a.cpu_budget)
+        out["cpu_baseline"] = {"value": round(ops / secs / 1e12, 8), "unit": unit, "cores": 1,
+                               "kind": "oracle",
+                               "sample": f"{rows} of {T} token rows of {W.config['workload']}, "
+                                         f"plain C oracle, single thread, {secs:.1f} s"}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main_reference(a, rank, world):
+    """The CPU oracle as the reference arm: rank 0 only, bounded samples."""
+    if rank != 0:
+        return 0
+    ops_tot, secs_tot, rows_tot = 0, 0.0, 0
+    per_step_budget = max(0.5, min(8.0, 120.0 / max(1, a.steps + a.warmup)))
+    T = 0
+    for i in range(a.warmup + a.steps):
+        ops, secs, rows, T = oracle_sample(a.workload, budget_s=per_step_budget, max_rows=64)
+        if i >= a.warmup:
+            ops_tot += ops
+            secs_tot += secs
+            rows_tot += rows
+    value = ops_tot / secs_tot / 1e12
+    metric = "W8A8 linear INT8 TOPS (whole step, incl. fused LN/token-quant)"
+    out = {"impl": "reference", "metric": metric, "value": round(value, 8), "unit": "TOPS",
+           "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+           "ms_per_step": round(1e3 * secs_tot / a.steps, 3), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+           "config": {"workload": a.workload, "sample_rows_per_step": rows_tot // max(1, a.steps),
+                      "total_rows": T},
+           "cpu_baseline": {"value": round(value, 8), "unit": "TOPS", "cores": 1, "kind": "oracle",
+                            "sample": f"{rows_tot // max(1, a.steps)} token rows per step of {T}"},
+           "e2e": {"value": round(value, 8), "unit": "TOPS", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,188 @@
+/*
+ * zq.h -- C ABI of the B200 (sm_100a) ZeroQuant-style W8A8 linear library.
+ *
+ * The hot path of W8A8 post-training-quantized inference, as three fused
+ * steps:
+ *   1. LayerNorm (or bias + GeLU) fused with dynamic per-token symmetric
+ *      INT8 quantization of the activations;
+ *   2. an INT8 x INT8 -> INT32 GEMM against weights quantized in groups of
+ *      contiguous output rows;
+ *   3. a dequantization epilogue fused into the GEMM:
+ *      y[t, o] = s_tok[t] * s_grp[o / G] * acc[t, o] + bias[o]
+ *      (+ GeLU, + per-token requantization for the next layer).
+ *
+ * Sources (web pages):
+ *   [ZQ]   "[2022 NeurIPS] ZeroQuant: Efficient and Affordable Post-Training
+ *          Quantization for Large-Scale Transformers": group-wise weight
+ *          quantization; token-wise activation quantization; the fused
+ *          kernel flowcharts "LN/GeLU + Quantize" and "GEMM + DeQuantize".
+ *   [TS36] "探秘Transformer系列之（36）— 大模型量化方案": §1.1.2 absmax
+ *          quantization to [-127, 127] and vector-wise scales; §1.2.2
+ *          per-token dynamic activation quantization fused with LayerNorm,
+ *          INT32 accumulators scaled by both scales before the next op,
+ *          group-wise weight quantization.
+ *   [IQ]   "Integer Quantization: Deep Dive": quantization formula with
+ *          clamp; dequantization x = s * x_int (zero-point 0 here).
+ *
+ * Numerics fixed by this library where the pages are silent:
+ *   scale = absmax / 127 (fp32 IEEE division); code = clamp(rint(v * (127 /
+ *   absmax)), -127, 127) with ties to even; an all-zero row or group has
+ *   scale 0 and codes 0; LayerNorm uses the biased variance, eps inside the
+ *   square root; GeLU is the erf form; bias is added after dequantization.
+ *
+ * Conventions for every entry point:
+ *   - Matrices are dense row-major; the leading dimension equals the row
+ *     length.  Activations are [T, K] (T tokens); weights are [N, K]
+ *     (N output features, the nn.Linear layout).
+ *   - Every pointer except where stated is a DEVICE pointer owned by the
+ *     caller; the library keeps no reference after the call returns and
+ *     allocates no device memory.  Scratch memory is passed in explicitly
+ *     as (workspace, workspace_bytes).
+ *   - Tensor pointers (x, q, Wq, W, y, workspace, gamma, beta) must be 16-byte
+ *     aligned; scale and bias vectors 4-byte aligned.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL means the legacy default stream).  They return a zq_status.
+ *     Arguments are validated on the host before anything is enqueued; a
+ *     call that returns an error has launched nothing.  No call aborts,
+ *     traps or prints.
+ *   - Device-side waits inside the GEMM are bounded.  If one expires the
+ *     kernel records the fact in a device flag and returns early (output
+ *     undefined); zq_device_status() reports it as ZQ_ERR_TIMEOUT.
+ *   - NaN or Inf inputs are outside the contract (not checked on device).
+ */
+#ifndef ZQ_H_
+#define ZQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+enum zq_status {
+    ZQ_OK = 0,
+    ZQ_ERR_NULL = 1,      /* a required pointer is NULL                         */
+    ZQ_ERR_SHAPE = 2,     /* dimension <= 0, not a multiple of 16, N % G != 0,
+                             or beyond a documented maximum                     */
+    ZQ_ERR_ALIGN = 3,     /* pointer misaligned (see conventions)               */
+    ZQ_ERR_OVERFLOW = 4,  /* K > ZQ_MAX_K: 127*127*K could leave int32          */
+    ZQ_ERR_DTYPE = 5,     /* unknown dtype / activation / output-kind enum      */
+    ZQ_ERR_CUDA = 6,      /* CUDA runtime/driver error; see zq_last_cuda_error  */
+    ZQ_ERR_TIMEOUT = 7,   /* a bounded device-side wait expired                 */
+    ZQ_ERR_WORKSPACE = 8, /* workspace NULL or smaller than required            */
+    ZQ_ERR_DEVICE = 9     /* current device is not sm_100 (B200 class)          */
+};
+
+/* ---- enums --------------------------------------------------------------- */
+enum zq_dtype { ZQ_F32 = 0, ZQ_BF16 = 1 };            /* activation input types */
+enum zq_act { ZQ_ACT_NONE = 0, ZQ_ACT_GELU = 1 };     /* GeLU = erf form        */
+enum zq_out_kind {
+    ZQ_OUT_F32 = 0,        /* y fp32 [T, N]                                        */
+    ZQ_OUT_BF16 = 1,       /* y bf16 [T, N], rounded to nearest even from fp32     */
+    ZQ_OUT_I8_REQUANT = 2, /* y int8 [T, N] + s_tok_out fp32 [T]: the epilogue
+                              output (after act) is quantized per token again      */
+    ZQ_OUT_I32_RAW = 3     /* y int32 [T, N]: the raw accumulators (debug/parity)  */
+};
+
+/* 127*127*K must stay inside int32: K <= floor((2^31-1)/16129). */
+#define ZQ_MAX_K 133144
+/* Longest row the fused LayerNorm/act quantizer keeps on chip. */
+#define ZQ_MAX_H 65536
+
+/* ---- offline weight quantization ----------------------------------------
+ * [ZQ] group-wise quantization; [TS36] §1.2.2 and §1.1.2 (absmax rule).
+ * W     : fp32 [N, K] device, row-major.
+ * group_rows (G) : rows per group; group g = rows g*G .. g*G+G-1, all K
+ *         columns, one scale per group.  N % G == 0.  G = 1 gives per-row
+ *         (vector-wise) scales, G = N a single per-tensor scale.
+ * Wq    : int8 [N, K] device (output).
+ * s_grp : fp32 [N / G] device (output): absmax_g / 127.
+ * Constraints: K % 16 == 0.  Errors: NULL, SHAPE, ALIGN, CUDA, DEVICE. */
+int zq_quantize_weights(const float* W, int64_t N, int64_t K, int64_t group_rows,
+                        int8_t* Wq, float* s_grp, void* stream);
+
+/* ---- fused LayerNorm + per-token quantization ----------------------------
+ * [ZQ] "LN + Quantize" fused kernel; [TS36] §1.2.2 (quantization fused with
+ * the preceding LayerNorm, one dynamic scale per token).
+ * x      : [T, H] device, dtype x_dtype (ZQ_F32 or ZQ_BF16).
+ * gamma, beta : fp32 [H] device.  eps : added to the variance.
+ * q      : int8 [T, H] device (output); s_tok : fp32 [T] device (output).
+ * y = (x - mean) / sqrt(var + eps) * gamma + beta per row (fp32), then
+ * s_tok = absmax(y)/127, q = clamp(rint(y * 127/absmax(y))).
+ * Constraints: H % 16 == 0, H <= ZQ_MAX_H.  Errors: NULL, SHAPE, ALIGN,
+ * DTYPE, CUDA, DEVICE. */
+int zq_ln_quant(const void* x, int x_dtype, int64_t T, int64_t H,
+                const float* gamma, const float* beta, float eps,
+                int8_t* q, float* s_tok, void* stream);
+
+/* ---- fused (bias +) activation + per-token quantization ------------------
+ * [ZQ] "GeLU + Quantize" fused kernel.  y = act(x + bias) per element in
+ * fp32 (bias optional: NULL skips it; act ZQ_ACT_NONE or ZQ_ACT_GELU), then
+ * the per-token quantizer of zq_ln_quant.  With no bias and no act the codes
+ * and scales are exactly those of the quantizer applied to fp32(x).
+ * Shapes, outputs, constraints and errors as zq_ln_quant. */
+int zq_act_quant(const void* x, int x_dtype, int64_t T, int64_t H,
+                 const float* bias, int act, int8_t* q, float* s_tok, void* stream);
+
+/* ---- W8A8 linear: INT8 GEMM + fused dequantization epilogue --------------
+ * [ZQ] "GEMM + DeQuantize"; [TS36] §1.2.2 (INT32 accumulators scaled by the
+ * weight and activation scales before the write to the next op) and §1.1.2
+ * (denormalisation by the outer product of row and column scales).
+ * xq     : int8 [T, K] device;  s_tok : fp32 [T] device.
+ * Wq     : int8 [N, K] device;  s_grp : fp32 [N / G] device.
+ * bias   : fp32 [N] device or NULL.  act : applied after the bias.
+ * out_kind selects y's type (see zq_out_kind).  s_tok_out : fp32 [T] device,
+ *          written only for ZQ_OUT_I8_REQUANT (else may be NULL).
+ * acc[t, o] = sum_k xq[t, k] * Wq[o, k] (exact int32, tcgen05 INT8 MMA);
+ * y[t, o] = act(s_tok[t] * s_grp[o / G] * acc[t, o] + bias[o]) in fp32.
+ * ZQ_OUT_I32_RAW stores acc itself and requires act == ZQ_ACT_NONE and
+ * bias == NULL.
+ * workspace : device scratch of at least zq_w8a8_linear_workspace(...)
+ *          bytes (may be NULL when that is 0).  Its contents on entry do not
+ *          matter; it is clobbered.
+ * Constraints: K % 16 == 0, N % 16 == 0, N % G == 0, K <= ZQ_MAX_K.
+ * Errors: NULL, SHAPE, ALIGN, OVERFLOW, DTYPE, WORKSPACE, CUDA, DEVICE. */
+size_t zq_w8a8_linear_workspace(int64_t T, int64_t K, int64_t N, int out_kind);
+int zq_w8a8_linear(const int8_t* xq, const float* s_tok, int64_t T, int64_t K,
+                   const int8_t* Wq, const float* s_grp, int64_t N, int64_t group_rows,
+                   const float* bias, int act, int out_kind,
+                   void* y, float* s_tok_out,
+                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---- one quantized linear layer from floating-point activations ----------
+ * [ZQ] fused flowchart, both kernels: x -> [LN + Quantize] -> [GEMM +
+ * DeQuantize].  gamma != NULL: zq_ln_quant(x, gamma, beta, eps); gamma ==
+ * NULL: zq_act_quant(x, NULL, ZQ_ACT_NONE) (beta and eps ignored).  Then
+ * zq_w8a8_linear with the remaining arguments.  The quantized activations
+ * live in the workspace (zq_linear_block_workspace bytes).
+ * Errors: the union of the two calls'. */
+size_t zq_linear_block_workspace(int64_t T, int64_t K, int64_t N, int out_kind);
+int zq_linear_block(const void* x, int x_dtype, int64_t T, int64_t K,
+                    const float* gamma, const float* beta, float eps,
+                    const int8_t* Wq, const float* s_grp, int64_t N, int64_t group_rows,
+                    const float* bias, int act, int out_kind, void* y, float* s_tok_out,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---- diagnostics ----------------------------------------------------------
+ * zq_device_status: synchronizes `stream`, then reads and clears the device
+ * flag that bounded waits set on expiry.  Returns ZQ_OK, ZQ_ERR_TIMEOUT or
+ * ZQ_ERR_CUDA.  Not callable during stream capture.
+ * zq_status_string: static text for a status code (never NULL).
+ * zq_last_cuda_error: text of the last CUDA error seen by this thread's
+ * calls (static storage, "no error" when none).
+ * zq_version: library version as 10000*major + 100*minor + patch.
+ * zq_launch_count: number of kernels this library has launched in this
+ * process (all devices, all threads); for accounting in benchmarks. */
+int zq_device_status(void* stream);
+const char* zq_status_string(int status);
+const char* zq_last_cuda_error(void);
+int zq_version(void);
+uint64_t zq_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZQ_H_ */

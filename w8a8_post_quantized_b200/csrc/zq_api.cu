@@ -1,0 +1,279 @@
+// zq_api.cu -- the C ABI declared in include/zq.h: argument validation (all
+// of it on the host, before anything is enqueued), per-device facts, the
+// device status word used by bounded waits, and the entry points.
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "zq_internal.cuh"
+
+#define ZQ_VERSION 100  // 0.1.0
+
+namespace zq {
+
+// Device status word: bounded waits record the site of an expired wait here.
+__device__ int g_status_word;
+
+static thread_local char t_last_error[256] = "no error";
+static std::atomic<uint64_t> g_launches{0};
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+void set_cuda_error(cudaError_t e) {
+    snprintf(t_last_error, sizeof(t_last_error), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+int cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return ZQ_OK;
+    set_cuda_error(e);
+    return ZQ_ERR_CUDA;
+}
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+bool g_have[kMaxDevices];
+DeviceInfo g_info[kMaxDevices];
+}  // namespace
+
+int device_info(DeviceInfo* out) {
+    int dev = -1;
+    int rc = cuda_status(cudaGetDevice(&dev));
+    if (rc) return rc;
+    if (dev < 0 || dev >= kMaxDevices) return ZQ_ERR_DEVICE;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_have[dev]) {
+        DeviceInfo di{};
+        if ((rc = cuda_status(cudaDeviceGetAttribute(&di.sm_count, cudaDevAttrMultiProcessorCount, dev))))
+            return rc;
+        if ((rc = cuda_status(cudaDeviceGetAttribute(&di.major, cudaDevAttrComputeCapabilityMajor, dev))))
+            return rc;
+        if ((rc = cuda_status(cudaDeviceGetAttribute(&di.minor, cudaDevAttrComputeCapabilityMinor, dev))))
+            return rc;
+        void* addr = nullptr;
+        if ((rc = cuda_status(cudaGetSymbolAddress(&addr, g_status_word)))) return rc;
+        di.status_word = static_cast<int*>(addr);
+        g_info[dev] = di;
+        g_have[dev] = true;
+    }
+    *out = g_info[dev];
+    // sm_100a code only runs on compute capability 10.0 parts
+    if (out->major != 10 || out->minor != 0) return ZQ_ERR_DEVICE;
+    return ZQ_OK;
+}
+
+}  // namespace zq
+
+using namespace zq;
+
+namespace {
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+int check_rows(const void* x, int x_dtype, int64_t T, int64_t H, const int8_t* q, const float* s_tok) {
+    if (!x || !q || !s_tok) return ZQ_ERR_NULL;
+    if (x_dtype != ZQ_F32 && x_dtype != ZQ_BF16) return ZQ_ERR_DTYPE;
+    if (T <= 0 || H <= 0 || H % 16 != 0 || H > ZQ_MAX_H) return ZQ_ERR_SHAPE;
+    if (T > (int64_t)1 << 31) return ZQ_ERR_SHAPE;
+    if (!aligned(x, 16) || !aligned(q, 16) || !aligned(s_tok, 4)) return ZQ_ERR_ALIGN;
+    return ZQ_OK;
+}
+
+constexpr size_t kWsAlign = 256;
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+size_t linear_ws_bytes(int64_t T, int64_t K, int64_t N, int out_kind) {
+    (void)K;
+    if (out_kind != ZQ_OUT_I8_REQUANT || T <= 0 || N <= 0) return 0;
+    // fp32 [T, N] epilogue output + [T] absmax words
+    return round_up((size_t)T * (size_t)N * sizeof(float), kWsAlign) + round_up((size_t)T * 4, kWsAlign);
+}
+
+int check_linear(const int8_t* xq, const float* s_tok, int64_t T, int64_t K, const int8_t* Wq,
+                 const float* s_grp, int64_t N, int64_t G, const float* bias, int act, int out_kind,
+                 void* y, float* s_tok_out, void* ws, size_t ws_bytes, bool check_x) {
+    if (check_x && (!xq || !s_tok)) return ZQ_ERR_NULL;
+    if (!Wq || !s_grp || !y) return ZQ_ERR_NULL;
+    if (out_kind < ZQ_OUT_F32 || out_kind > ZQ_OUT_I32_RAW) return ZQ_ERR_DTYPE;
+    if (act != ZQ_ACT_NONE && act != ZQ_ACT_GELU) return ZQ_ERR_DTYPE;
+    if (out_kind == ZQ_OUT_I32_RAW && (act != ZQ_ACT_NONE || bias)) return ZQ_ERR_DTYPE;
+    if (out_kind == ZQ_OUT_I8_REQUANT && !s_tok_out) return ZQ_ERR_NULL;
+    if (T <= 0 || K <= 0 || N <= 0 || G <= 0) return ZQ_ERR_SHAPE;
+    if (K % 16 != 0 || N % 16 != 0 || N % G != 0) return ZQ_ERR_SHAPE;
+    if (T > (1 << 30) || N > (1 << 30)) return ZQ_ERR_SHAPE;
+    if (K > ZQ_MAX_K) return ZQ_ERR_OVERFLOW;
+    if (check_x && (!aligned(xq, 16) || !aligned(s_tok, 4))) return ZQ_ERR_ALIGN;
+    if (!aligned(Wq, 16) || !aligned(y, 16) || !aligned(s_grp, 4)) return ZQ_ERR_ALIGN;
+    if ((bias && !aligned(bias, 4)) || (s_tok_out && !aligned(s_tok_out, 4))) return ZQ_ERR_ALIGN;
+    const size_t need = linear_ws_bytes(T, K, N, out_kind);
+    if (need) {
+        if (!ws || ws_bytes < need) return ZQ_ERR_WORKSPACE;
+        if (!aligned(ws, 16)) return ZQ_ERR_ALIGN;
+    }
+    return ZQ_OK;
+}
+
+int run_linear(const int8_t* xq, const float* s_tok, int64_t T, int64_t K, const int8_t* Wq,
+               const float* s_grp, int64_t N, int64_t G, const float* bias, int act, int out_kind,
+               void* y, float* s_tok_out, void* ws, const DeviceInfo& di, cudaStream_t st) {
+    LinearArgs a{};
+    a.xq = xq;
+    a.s_tok = s_tok;
+    a.T = T;
+    a.K = K;
+    a.Wq = Wq;
+    a.s_grp = s_grp;
+    a.N = N;
+    a.G = G;
+    a.bias = bias;
+    a.act = act;
+    a.out_kind = out_kind;
+    a.y = y;
+    int rc;
+    if (out_kind == ZQ_OUT_I8_REQUANT) {
+        uint8_t* w = static_cast<uint8_t*>(ws);
+        a.h_ws = reinterpret_cast<float*>(w);
+        a.amax_ws = reinterpret_cast<uint32_t*>(w + round_up((size_t)T * N * sizeof(float), kWsAlign));
+        if ((rc = cuda_status(cudaMemsetAsync(a.amax_ws, 0, (size_t)T * 4, st)))) return rc;
+        if ((rc = launch_w8a8_gemm(a, di, st))) return rc;
+        return launch_requant_rows(a.h_ws, T, N, a.amax_ws, static_cast<int8_t*>(y), s_tok_out, di, st);
+    }
+    return launch_w8a8_gemm(a, di, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int zq_version(void) { return ZQ_VERSION; }
+
+uint64_t zq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* zq_status_string(int status) {
+    switch (status) {
+        case ZQ_OK: return "ok";
+        case ZQ_ERR_NULL: return "required pointer is NULL";
+        case ZQ_ERR_SHAPE: return "invalid shape (non-positive, not a multiple of 16, N % G != 0, or too large)";
+        case ZQ_ERR_ALIGN: return "misaligned pointer (tensors need 16 bytes, vectors 4 bytes)";
+        case ZQ_ERR_OVERFLOW: return "K too large: int32 accumulators could overflow";
+        case ZQ_ERR_DTYPE: return "unknown or unsupported dtype / activation / output kind";
+        case ZQ_ERR_CUDA: return "CUDA error (see zq_last_cuda_error)";
+        case ZQ_ERR_TIMEOUT: return "a bounded device-side wait expired";
+        case ZQ_ERR_WORKSPACE: return "workspace missing or too small";
+        case ZQ_ERR_DEVICE: return "current device is not an sm_100 (B200-class) GPU";
+        default: return "unknown status";
+    }
+}
+
+const char* zq_last_cuda_error(void) { return t_last_error; }
+
+int zq_device_status(void* stream) {
+    DeviceInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    if ((rc = cuda_status(cudaStreamSynchronize(as_stream(stream))))) return rc;
+    int word = 0;
+    if ((rc = cuda_status(cudaMemcpyFromSymbol(&word, g_status_word, sizeof(int))))) return rc;
+    if (word != 0) {
+        const int zero = 0;
+        if ((rc = cuda_status(cudaMemcpyToSymbol(g_status_word, &zero, sizeof(int))))) return rc;
+        snprintf(t_last_error, sizeof(t_last_error), "bounded wait expired at site 0x%x", word);
+        return ZQ_ERR_TIMEOUT;
+    }
+    return ZQ_OK;
+}
+
+int zq_quantize_weights(const float* W, int64_t N, int64_t K, int64_t group_rows, int8_t* Wq,
+                        float* s_grp, void* stream) {
+    if (!W || !Wq || !s_grp) return ZQ_ERR_NULL;
+    if (N <= 0 || K <= 0 || group_rows <= 0 || K % 16 != 0 || N % group_rows != 0) return ZQ_ERR_SHAPE;
+    if (N > ((int64_t)1 << 40) / K) return ZQ_ERR_SHAPE;
+    if (!aligned(W, 16) || !aligned(Wq, 16) || !aligned(s_grp, 4)) return ZQ_ERR_ALIGN;
+    DeviceInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    return launch_quantize_weights(W, N, K, group_rows, Wq, s_grp, di, as_stream(stream));
+}
+
+int zq_ln_quant(const void* x, int x_dtype, int64_t T, int64_t H, const float* gamma,
+                const float* beta, float eps, int8_t* q, float* s_tok, void* stream) {
+    int rc = check_rows(x, x_dtype, T, H, q, s_tok);
+    if (rc) return rc;
+    if (!gamma || !beta) return ZQ_ERR_NULL;
+    if (!aligned(gamma, 16) || !aligned(beta, 16)) return ZQ_ERR_ALIGN;
+    if (!(eps >= 0.0f)) return ZQ_ERR_SHAPE;
+    DeviceInfo di;
+    if ((rc = device_info(&di))) return rc;
+    return launch_ln_quant(x, x_dtype, T, H, gamma, beta, eps, q, s_tok, di, as_stream(stream));
+}
+
+int zq_act_quant(const void* x, int x_dtype, int64_t T, int64_t H, const float* bias, int act,
+                 int8_t* q, float* s_tok, void* stream) {
+    int rc = check_rows(x, x_dtype, T, H, q, s_tok);
+    if (rc) return rc;
+    if (act != ZQ_ACT_NONE && act != ZQ_ACT_GELU) return ZQ_ERR_DTYPE;
+    if (bias && !aligned(bias, 16)) return ZQ_ERR_ALIGN;
+    DeviceInfo di;
+    if ((rc = device_info(&di))) return rc;
+    return launch_act_quant(x, x_dtype, T, H, bias, act, q, s_tok, di, as_stream(stream));
+}
+
+size_t zq_w8a8_linear_workspace(int64_t T, int64_t K, int64_t N, int out_kind) {
+    return linear_ws_bytes(T, K, N, out_kind);
+}
+
+int zq_w8a8_linear(const int8_t* xq, const float* s_tok, int64_t T, int64_t K, const int8_t* Wq,
+                   const float* s_grp, int64_t N, int64_t group_rows, const float* bias, int act,
+                   int out_kind, void* y, float* s_tok_out, void* workspace, size_t workspace_bytes,
+                   void* stream) {
+    int rc = check_linear(xq, s_tok, T, K, Wq, s_grp, N, group_rows, bias, act, out_kind, y, s_tok_out,
+                          workspace, workspace_bytes, true);
+    if (rc) return rc;
+    DeviceInfo di;
+    if ((rc = device_info(&di))) return rc;
+    return run_linear(xq, s_tok, T, K, Wq, s_grp, N, group_rows, bias, act, out_kind, y, s_tok_out,
+                      workspace, di, as_stream(stream));
+}
+
+size_t zq_linear_block_workspace(int64_t T, int64_t K, int64_t N, int out_kind) {
+    if (T <= 0 || K <= 0) return 0;
+    return round_up((size_t)T * (size_t)K, kWsAlign) + round_up((size_t)T * 4, kWsAlign) +
+           linear_ws_bytes(T, K, N, out_kind);
+}
+
+int zq_linear_block(const void* x, int x_dtype, int64_t T, int64_t K, const float* gamma,
+                    const float* beta, float eps, const int8_t* Wq, const float* s_grp, int64_t N,
+                    int64_t group_rows, const float* bias, int act, int out_kind, void* y,
+                    float* s_tok_out, void* workspace, size_t workspace_bytes, void* stream) {
+    if (!x) return ZQ_ERR_NULL;
+    if (x_dtype != ZQ_F32 && x_dtype != ZQ_BF16) return ZQ_ERR_DTYPE;
+    if (T <= 0 || K <= 0 || K > ZQ_MAX_H) return ZQ_ERR_SHAPE;
+    if (gamma && !beta) return ZQ_ERR_NULL;
+    if (gamma && (!aligned(gamma, 16) || !aligned(beta, 16))) return ZQ_ERR_ALIGN;
+    if (gamma && !(eps >= 0.0f)) return ZQ_ERR_SHAPE;
+    if (!aligned(x, 16)) return ZQ_ERR_ALIGN;
+    const size_t need = zq_linear_block_workspace(T, K, N, out_kind);
+    if (!workspace || workspace_bytes < need) return ZQ_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return ZQ_ERR_ALIGN;
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    int8_t* xq = reinterpret_cast<int8_t*>(w);
+    float* s_tok = reinterpret_cast<float*>(w + round_up((size_t)T * K, kWsAlign));
+    uint8_t* lin_ws = w + round_up((size_t)T * K, kWsAlign) + round_up((size_t)T * 4, kWsAlign);
+    const size_t lin_bytes = workspace_bytes - (size_t)(lin_ws - w);
+    int rc = check_linear(xq, s_tok, T, K, Wq, s_grp, N, group_rows, bias, act, out_kind, y, s_tok_out,
+                          lin_ws, lin_bytes, false);
+    if (rc) return rc;
+    DeviceInfo di;
+    if ((rc = device_info(&di))) return rc;
+    cudaStream_t st = as_stream(stream);
+    if (gamma) rc = launch_ln_quant(x, x_dtype, T, K, gamma, beta, eps, xq, s_tok, di, st);
+    else rc = launch_act_quant(x, x_dtype, T, K, nullptr, ZQ_ACT_NONE, xq, s_tok, di, st);
+    if (rc) return rc;
+    return run_linear(xq, s_tok, T, K, Wq, s_grp, N, group_rows, bias, act, out_kind, y, s_tok_out,
+                      lin_ws, di, st);
+}
+
+}  // extern "C"

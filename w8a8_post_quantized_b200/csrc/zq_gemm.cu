@@ -1,0 +1,462 @@
+// zq_gemm.cu -- W8A8 linear for sm_100a: INT8 x INT8 -> INT32 on the
+// 5th-generation tensor cores (tcgen05.mma kind::i8) with the
+// dequantization epilogue fused.
+//
+// Sources: "[2022 NeurIPS] ZeroQuant: Efficient and Affordable Post-Training
+// Quantization for Large-Scale Transformers" (the fused "GEMM + DeQuantize"
+// kernel) and "探秘Transformer系列之（36）— 大模型量化方案" §1.2.2 (the INT32
+// accumulation is scaled by the activation and weight scales before the
+// result is written for the next op) and §1.1.2 (denormalisation by the outer
+// product of the per-row and per-column scales).  The pages' kernel targets
+// Ampere (WMMA tiles via CUTLASS, group size tuned to 16/32); here groups are
+// whole output rows, so the scale of an output column is constant along K and
+// the whole contraction stays in exact int32 on the tensor core, with the
+// scales applied once per output element in the epilogue.
+//
+// Structure (one persistent CTA per SM, 6 warps):
+//   warp 0      TMA producer: 128-row x 128-byte tiles of both operands into
+//               a STAGES-deep shared-memory ring (128-byte swizzle), one
+//               mbarrier per stage counting the bytes that landed;
+//   warp 1      allocates TMEM, then one thread issues tcgen05.mma (M=128,
+//               N=BN, K=32 per instruction, 4 per stage) into one of two
+//               TMEM accumulators and commits stage release / tile-done
+//               mbarriers;
+//   warps 2..5  epilogue: tcgen05.ld of the int32 accumulator (each warp
+//               owns its 32-lane quarter of TMEM), dequantize with the
+//               token and group scales, add bias, optional GeLU, store
+//               fp32 / bf16 / int32, or fp32 plus a per-row absmax for
+//               requantization.  Two accumulators let the epilogue of tile
+//               i overlap the main loop of tile i+1.
+// Operand roles: normally the M side is the activations (rows = tokens) and
+// the N side the weights; for few tokens (decode) the roles swap so the
+// weights fill the 128-row MMA side and the tokens become N = 16..64.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "zq_internal.cuh"
+
+namespace zq {
+namespace {
+
+constexpr int BM = 128;         // MMA M: rows of the M-side operand per tile
+constexpr int BK = 128;         // K bytes per pipeline stage (one swizzle row)
+constexpr int UMMA_K = 32;      // K per tcgen05.mma of kind::i8
+constexpr int kThreads = 192;   // 6 warps
+constexpr int kEpiThreads = 128;
+constexpr int A_STAGE = BM * BK;
+
+enum Epi { EPI_I32 = 0, EPI_F32 = 1, EPI_BF16 = 2, EPI_REQ = 3 };
+
+// Status sites recorded when a bounded wait expires.
+enum WaitSite {
+    SITE_PRODUCER_EMPTY = 0x101,
+    SITE_MMA_TMEM_EMPTY = 0x201,
+    SITE_MMA_FULL = 0x202,
+    SITE_MMA_DRAIN = 0x203,
+    SITE_EPI_TMEM_FULL = 0x301,
+    SITE_PRODUCER_DRAIN = 0x102,
+};
+
+struct Params {
+    int M, N, K;        // kernel roles: M-side rows, N-side rows, reduction length
+    int G;              // weight rows per scale group
+    int ldy;            // row length of y (= number of output features)
+    const float* s_tok;
+    const float* s_grp;
+    const float* bias;  // may be null
+    void* y;
+    uint32_t* amax;     // EPI_REQ: per-token absmax bits
+    int act;
+    int* status;
+};
+
+template <int BN>
+constexpr uint32_t tmem_cols() {
+    return (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128 : (2 * BN <= 256) ? 256 : 512;
+}
+
+template <int BN, int STAGES>
+constexpr size_t smem_bytes() {
+    // 1024 alignment slack + operand ring + barriers/flags + epilogue staging
+    return 1024 + (size_t)STAGES * (A_STAGE + BN * BK) + 256 + 2 * BN * sizeof(float);
+}
+
+template <int BN, int STAGES, bool SWAP, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const Params p) {
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128 is 16..256 step 16");
+    constexpr int B_STAGE = BN * BK;
+    constexpr int CW = (BN % 32 == 0) ? 32 : 16;  // epilogue column chunk
+    constexpr uint32_t IDESC = idesc_i8(BM, BN);
+    constexpr uint32_t TMEM_COLS = tmem_cols<BN>();
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - raw);
+    const uint32_t sA = base;
+    const uint32_t sB = base + STAGES * A_STAGE;
+    const uint32_t sBar = sB + STAGES * B_STAGE;
+    uint8_t* gBar = gbase + (sBar - base);
+    // barrier layout: full[S], empty[S], tfull[2], tempty[2], drain
+    auto bar_full = [&](int s) { return sBar + 8u * s; };
+    auto bar_empty = [&](int s) { return sBar + 8u * (STAGES + s); };
+    auto bar_tfull = [&](int b) { return sBar + 8u * (2 * STAGES + b); };
+    auto bar_tempty = [&](int b) { return sBar + 8u * (2 * STAGES + 2 + b); };
+    const uint32_t bar_drain = sBar + 8u * (2 * STAGES + 4);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gBar + 8 * (2 * STAGES + 5));
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    float* stage_f = reinterpret_cast<float*>(gBar + 256);  // [2][BN]
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(bar_full(s), 1);
+            mbar_init(bar_empty(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar_tfull(b), 1);
+            mbar_init(bar_tempty(b), kEpiThreads / 32);
+        }
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        fence_proxy_async_smem();
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int m_tiles = (p.M + BM - 1) / BM;
+    const int n_tiles = (p.N + BN - 1) / BN;
+    const int num_tiles = m_tiles * n_tiles;
+    const int kblocks = (p.K + BK - 1) / BK;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+                const int mt = tile % m_tiles, nt = tile / m_tiles;
+                for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1u;
+                    if (!mbar_wait(bar_empty(s), ph ^ 1u, abort_flag, p.status, SITE_PRODUCER_EMPTY)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(bar_full(s), A_STAGE + B_STAGE);
+                    tma_load_2d(sA + s * A_STAGE, &tmA, bar_full(s), kb * BK, mt * BM);
+                    tma_load_2d(sB + s * B_STAGE, &tmB, bar_full(s), kb * BK, nt * BN);
+                }
+            }
+            // Let every copy this thread issued land before the CTA can exit:
+            // wait on the most recent phase of each stage that was used.
+            const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0u;
+            for (uint32_t j = first; j < it; ++j)
+                mbar_wait(bar_full(j % STAGES), (j / STAGES) & 1u, nullptr, p.status,
+                          SITE_PRODUCER_DRAIN);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint32_t it = 0, lt = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++lt) {
+                const int b = lt & 1;
+                const uint32_t tph = (lt >> 1) & 1u;
+                if (!mbar_wait(bar_tempty(b), tph ^ 1u, abort_flag, p.status, SITE_MMA_TMEM_EMPTY)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(b * BN);
+                for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1u;
+                    if (!mbar_wait(bar_full(s), ph, abort_flag, p.status, SITE_MMA_FULL)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t da = sdesc_k_sw128(sA + s * A_STAGE);
+                    const uint64_t db = sdesc_k_sw128(sB + s * B_STAGE);
+#pragma unroll
+                    for (int k = 0; k < BK / UMMA_K; ++k)
+                        // +32 bytes along K inside the swizzle atom = +2 in the
+                        // descriptor's (address >> 4) field
+                        mma_i8(d_tmem, da + 2u * k, db + 2u * k, IDESC, (kb | k) != 0 ? 1u : 0u);
+                    mma_commit(bar_empty(s));  // stage free once these MMAs finish
+                }
+                if (ok) mma_commit(bar_tfull(b));  // accumulator b complete
+            }
+            // All MMAs issued by this thread complete before teardown.
+            mma_commit(bar_drain);
+            mbar_wait(bar_drain, 0u, nullptr, p.status, SITE_MMA_DRAIN);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ epilogue
+        const int quarter = warp & 3;           // TMEM lanes 32*quarter .. +31
+        const int r = quarter * 32 + lane;      // row of the tile this thread owns
+        const int et = threadIdx.x - 64;        // 0..127
+        float* st_a = stage_f;                  // per-column scale (or token scale when swapped)
+        float* st_b = stage_f + BN;             // per-column bias (non-swapped)
+        uint32_t lt = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++lt) {
+            const int mt = tile % m_tiles, nt = tile / m_tiles;
+            const int b = lt & 1;
+            const uint32_t tph = (lt >> 1) & 1u;
+            // stage the per-column factors of this tile (previous readers done)
+            named_bar_sync(1, kEpiThreads);
+            for (int i = et; i < BN; i += kEpiThreads) {
+                const int n = nt * BN + i;
+                const bool in = n < p.N;
+                if constexpr (SWAP) {
+                    st_a[i] = (EPI != EPI_I32 && in) ? __ldg(p.s_tok + n) : 0.0f;
+                } else {
+                    st_a[i] = (EPI != EPI_I32 && in) ? __ldg(p.s_grp + n / p.G) : 0.0f;
+                    st_b[i] = (EPI != EPI_I32 && in && p.bias) ? __ldg(p.bias + n) : 0.0f;
+                }
+            }
+            named_bar_sync(1, kEpiThreads);
+            // all 128 epilogue threads take the same decision (barrier with an
+            // AND-reduction), so none is left behind at a later barrier
+            const bool got = mbar_wait(bar_tfull(b), tph, abort_flag, p.status, SITE_EPI_TMEM_FULL);
+            if (!named_bar_and(1, kEpiThreads, got)) break;
+            tc_fence_after();
+
+            const int gm = mt * BM + r;          // M-side row owned by this thread
+            const bool row_ok = gm < p.M;
+            float row_scale = 0.0f, row_bias = 0.0f;
+            if (EPI != EPI_I32 && row_ok) {
+                if constexpr (SWAP) {
+                    row_scale = __ldg(p.s_grp + gm / p.G);
+                    row_bias = p.bias ? __ldg(p.bias + gm) : 0.0f;
+                } else {
+                    row_scale = __ldg(p.s_tok + gm);
+                }
+            }
+            float amax = 0.0f;
+            const uint32_t t_row = tmem_base + (uint32_t)(b * BN) + ((uint32_t)(quarter * 32) << 16);
+
+#pragma unroll 1
+            for (int c = 0; c < BN / CW; ++c) {
+                uint32_t v[CW];
+                if constexpr (CW == 32) tmem_ld_32x32b_x32(t_row + c * CW, v);
+                else tmem_ld_32x32b_x16(t_row + c * CW, v);
+                tmem_ld_wait();
+                const int n0 = nt * BN + c * CW;   // first N-side index of the chunk
+                if constexpr (!SWAP) {
+                    // thread owns token gm, columns n0 .. n0+CW-1 (output features)
+                    if (!row_ok) continue;
+#pragma unroll
+                    for (int h = 0; h < CW / 16; ++h) {
+                        const int nb = n0 + 16 * h;
+                        if (nb >= p.N) break;      // N % 16 == 0: 16-column groups are whole
+                        const int64_t off = (int64_t)gm * p.ldy + nb;
+                        if constexpr (EPI == EPI_I32) {
+                            int4* dst = reinterpret_cast<int4*>(static_cast<int32_t*>(p.y) + off);
+#pragma unroll
+                            for (int q4 = 0; q4 < 4; ++q4)
+                                dst[q4] = make_int4((int)v[16 * h + 4 * q4], (int)v[16 * h + 4 * q4 + 1],
+                                                    (int)v[16 * h + 4 * q4 + 2], (int)v[16 * h + 4 * q4 + 3]);
+                        } else {
+                            float yv[16];
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                const int i = c * CW + 16 * h + j;
+                                float t = fmaf(row_scale * st_a[i], (float)(int)v[16 * h + j], st_b[i]);
+                                if (p.act == ZQ_ACT_GELU) t = gelu_f(t);
+                                yv[j] = t;
+                            }
+                            if constexpr (EPI == EPI_BF16) {
+                                uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.y) + off);
+#pragma unroll
+                                for (int q8 = 0; q8 < 2; ++q8)
+                                    dst[q8] = make_uint4(pack_bf16x2(yv[8 * q8 + 0], yv[8 * q8 + 1]),
+                                                         pack_bf16x2(yv[8 * q8 + 2], yv[8 * q8 + 3]),
+                                                         pack_bf16x2(yv[8 * q8 + 4], yv[8 * q8 + 5]),
+                                                         pack_bf16x2(yv[8 * q8 + 6], yv[8 * q8 + 7]));
+                            } else {
+                                float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.y) + off);
+#pragma unroll
+                                for (int q4 = 0; q4 < 4; ++q4)
+                                    dst[q4] = make_float4(yv[4 * q4], yv[4 * q4 + 1], yv[4 * q4 + 2],
+                                                          yv[4 * q4 + 3]);
+                                if constexpr (EPI == EPI_REQ) {
+#pragma unroll
+                                    for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(yv[j]));
+                                }
+                            }
+                        }
+                    }
+                } else {
+                    // thread owns output feature gm, columns = tokens n0 .. n0+CW-1
+#pragma unroll
+                    for (int j = 0; j < CW; ++j) {
+                        const int tok = n0 + j;
+                        float t = 0.0f;
+                        if (EPI != EPI_I32) {
+                            t = fmaf(row_scale * st_a[c * CW + j], (float)(int)v[j], row_bias);
+                            if (p.act == ZQ_ACT_GELU) t = gelu_f(t);
+                        }
+                        if (EPI == EPI_REQ) {
+                            // absmax over this warp's 32 features, one atomic per token
+                            float m = (row_ok && tok < p.N) ? fabsf(t) : 0.0f;
+#pragma unroll
+                            for (int o = 16; o > 0; o >>= 1)
+                                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+                            if (lane == 0 && tok < p.N) atomicMax(p.amax + tok, __float_as_uint(m));
+                        }
+                        if (!row_ok || tok >= p.N) continue;
+                        const int64_t off = (int64_t)tok * p.ldy + gm;
+                        if constexpr (EPI == EPI_I32) static_cast<int32_t*>(p.y)[off] = (int32_t)v[j];
+                        else if constexpr (EPI == EPI_BF16)
+                            static_cast<__nv_bfloat16*>(p.y)[off] = __float2bfloat16_rn(t);
+                        else static_cast<float*>(p.y)[off] = t;
+                    }
+                }
+            }
+            // accumulator b may be overwritten once all four warps have read it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_tempty(b));
+            if constexpr (EPI == EPI_REQ && !SWAP) {
+                if (row_ok) atomicMax(p.amax + gm, __float_as_uint(amax));
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+// ------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// int8 matrix [rows, K] row-major; box = 128 bytes of K x box_rows rows,
+// 128-byte swizzle (matches sdesc_k_sw128); out-of-range elements read as 0.
+int make_tmap_i8(CUtensorMap* tm, const void* ptr, int64_t rows, int64_t K, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return ZQ_ERR_CUDA;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K};
+    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box,
+                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ZQ_OK : ZQ_ERR_CUDA;
+}
+
+constexpr int kMaxDevices = 64;
+
+template <int BN, int STAGES, bool SWAP, int EPI>
+int launch_cfg(const CUtensorMap& ta, const CUtensorMap& tb, const Params& p, const DeviceInfo& di,
+               cudaStream_t st) {
+    static_assert(smem_bytes<BN, STAGES>() <= 232448, "shared memory budget");
+    static_assert(smem_bytes<BN, STAGES>() > 116 * 1024, "one CTA per SM (TMEM ownership)");
+    auto kern = w8a8_gemm_kernel<BN, STAGES, SWAP, EPI>;
+    static bool attr_set[kMaxDevices] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= kMaxDevices) return ZQ_ERR_DEVICE;
+    if (!attr_set[dev]) {
+        int rc = cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  (int)smem_bytes<BN, STAGES>()));
+        if (rc) return rc;
+        attr_set[dev] = true;
+    }
+    const int tiles = ((p.M + BM - 1) / BM) * ((p.N + BN - 1) / BN);
+    const int grid = tiles < di.sm_count ? tiles : di.sm_count;
+    count_launch();
+    kern<<<grid, kThreads, smem_bytes<BN, STAGES>(), st>>>(ta, tb, p);
+    return cuda_status(cudaGetLastError());
+}
+
+template <int BN, int STAGES, bool SWAP>
+int launch_epi(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const Params& p,
+               const DeviceInfo& di, cudaStream_t st) {
+    switch (epi) {
+        case EPI_I32: return launch_cfg<BN, STAGES, SWAP, EPI_I32>(ta, tb, p, di, st);
+        case EPI_F32: return launch_cfg<BN, STAGES, SWAP, EPI_F32>(ta, tb, p, di, st);
+        case EPI_BF16: return launch_cfg<BN, STAGES, SWAP, EPI_BF16>(ta, tb, p, di, st);
+        default: return launch_cfg<BN, STAGES, SWAP, EPI_REQ>(ta, tb, p, di, st);
+    }
+}
+
+}  // namespace
+
+int launch_w8a8_gemm(const LinearArgs& a, const DeviceInfo& di, cudaStream_t st) {
+    int epi;
+    switch (a.out_kind) {
+        case ZQ_OUT_F32: epi = EPI_F32; break;
+        case ZQ_OUT_BF16: epi = EPI_BF16; break;
+        case ZQ_OUT_I8_REQUANT: epi = EPI_REQ; break;
+        default: epi = EPI_I32; break;
+    }
+    Params p{};
+    p.K = (int)a.K;
+    p.G = (int)a.G;
+    p.ldy = (int)a.N;
+    p.s_tok = a.s_tok;
+    p.s_grp = a.s_grp;
+    p.bias = a.bias;
+    p.y = epi == EPI_REQ ? static_cast<void*>(a.h_ws) : a.y;
+    p.amax = a.amax_ws;
+    p.act = a.act;
+    p.status = di.status_word;
+
+    const bool swap = a.T <= 64;
+    CUtensorMap ta, tb;
+    int rc;
+    if (swap) {
+        // M side = weights [N, K]; N side = tokens [T, K], BN = T rounded up to 16 (<= 64)
+        p.M = (int)a.N;
+        p.N = (int)a.T;
+        const int bn = a.T <= 16 ? 16 : a.T <= 32 ? 32 : 64;
+        if ((rc = make_tmap_i8(&ta, a.Wq, a.N, a.K, BM))) return rc;
+        if ((rc = make_tmap_i8(&tb, a.xq, a.T, a.K, bn))) return rc;
+        if (bn == 16) return launch_epi<16, 8, true>(epi, ta, tb, p, di, st);
+        if (bn == 32) return launch_epi<32, 8, true>(epi, ta, tb, p, di, st);
+        return launch_epi<64, 8, true>(epi, ta, tb, p, di, st);
+    }
+    p.M = (int)a.T;
+    p.N = (int)a.N;
+    const int bn = a.N >= 256 ? 256 : 128;
+    if ((rc = make_tmap_i8(&ta, a.xq, a.T, a.K, BM))) return rc;
+    if ((rc = make_tmap_i8(&tb, a.Wq, a.N, a.K, bn))) return rc;
+    if (bn == 256) return launch_epi<256, 4, false>(epi, ta, tb, p, di, st);
+    return launch_epi<128, 6, false>(epi, ta, tb, p, di, st);
+}
+
+}  // namespace zq
