@@ -15,9 +15,11 @@ ops per GEMM, summed, over the step time), with the fused LN/token-quant
 bandwidth and the per-kernel roofline alongside.
 
 Timing: each stage is one CUDA graph of the library's C-ABI calls; every
-timed step is preceded by a 256 MiB write that flushes the 126 MB L2 and is
-bracketed by CUDA events on the launching stream (the flush is outside the
-events).  W >= 3 warm-up steps; K timed steps; barrier + synchronize on both
+timed step is preceded by an L2 flush -- a 256 MiB write followed by a read
+of the same buffer, so the 126 MB L2 ends up holding only clean lines of the
+flush buffer and no write-back of flush data lands inside the timed step --
+and is bracketed by CUDA events on the launching stream (the flush is
+outside the events).  W >= 3 warm-up steps; K timed steps; barrier + synchronize on both
 sides; the maximum over ranks.  Multi-GPU runs are independent replicas
 (the path needs no exchange): value = ops of all ranks / max time.
 
@@ -49,6 +51,18 @@ SPEC_INT8_TOPS = 4500.0          # dense INT8 tensor-core peak, spec
 SPEC_HBM_GBS = 8000.0
 INT8_OVER_BF16 = 2.0             # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 L2_FLUSH_BYTES = 256 << 20
+
+
+class L2Flush:
+    """Write then read back a buffer twice the size of L2 (leaves L2 clean)."""
+
+    def __init__(self, torch, device):
+        self.buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=device)
+        self.sink = torch.empty(1, dtype=torch.int32, device=device)
+
+    def __call__(self):
+        self.buf.fill_(1)
+        self.sink.copy_(self.buf.max().view(1))
 
 
 def load_peaks():
@@ -255,7 +269,7 @@ def time_device(W, steps, warmup, torch):
     """Per-stage CUDA graphs; flush L2 before each step; CUDA events around
     each stage on the launching stream.  Returns per-step and per-stage ms."""
     stream = torch.cuda.current_stream()
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=W.device)
+    flush = L2Flush(torch, W.device)
     for _, fn in W.stages:       # eager warm-up (sets kernel attributes, loads modules)
         fn()
     torch.cuda.synchronize()
@@ -275,7 +289,7 @@ def time_device(W, steps, warmup, torch):
     def run(k, record):
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(k)]
         for s in range(k):
-            flush.zero_()
+            flush()
             evs[s][0].record(stream)
             for i, (_, g) in enumerate(graphs):
                 g.replay()
@@ -304,7 +318,7 @@ def time_e2e(W, steps, warmup, torch):
     host_in.copy_(src.cpu())
     out = W.out
     host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=W.device)
+    flush = L2Flush(torch, W.device)
 
     def step():
         src.copy_(host_in, non_blocking=True)
@@ -313,12 +327,12 @@ def time_e2e(W, steps, warmup, torch):
         host_out.copy_(out, non_blocking=True)
 
     for _ in range(warmup):
-        flush.zero_()
+        flush()
         step()
     torch.cuda.synchronize()
     times = []
     for _ in range(steps):
-        flush.zero_()
+        flush()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
@@ -470,7 +484,7 @@ def main(argv=None):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
         "data": "synthetic (seeded; layer shapes only, random weights)",
         "config": dict(W.config, parallelism=f"replicas x{world}",
-                       l2="flushed (256 MiB write) before every timed step",
+                       l2="flushed before every timed step (256 MiB write + read-back)",
                        timing="per-stage CUDA graphs, CUDA events on the launching stream"),
         "tokens_per_s": round(world * W.tokens / (ms_per_step * 1e-3), 1),
         "stages_ms": {k: round(v, 5) for k, v in stage_ms.items()},
