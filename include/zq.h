@@ -72,7 +72,9 @@ enum zq_status {
     ZQ_ERR_CUDA = 6,      /* CUDA runtime/driver error; see zq_last_cuda_error  */
     ZQ_ERR_TIMEOUT = 7,   /* a bounded device-side wait expired                 */
     ZQ_ERR_WORKSPACE = 8, /* workspace NULL or smaller than required            */
-    ZQ_ERR_DEVICE = 9     /* current device is not sm_100 (B200 class)          */
+    ZQ_ERR_DEVICE = 9,    /* current device is not sm_100 (B200 class)          */
+    ZQ_ERR_SCRATCH = 10   /* problem larger than the fixed scratch array of
+                             zq_w8a8_linear_requant_noalloc                      */
 };
 
 /* ---- enums --------------------------------------------------------------- */
@@ -164,6 +166,37 @@ int zq_linear_block(const void* x, int x_dtype, int64_t T, int64_t K,
                     const int8_t* Wq, const float* s_grp, int64_t N, int64_t group_rows,
                     const float* bias, int act, int out_kind, void* y, float* s_tok_out,
                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---- requantizing linear without caller scratch ---------------------------
+ * No counterpart on the source pages: this entry point exists for callers,
+ * not for the method.  It computes exactly what zq_w8a8_linear computes with
+ * out_kind = ZQ_OUT_I8_REQUANT (same kernels, same results), but takes no
+ * workspace and allocates nothing.
+ *
+ * Who needs it: callers that cannot obtain device memory themselves -- code
+ * running inside a host framework that owns every device allocation and
+ * gives its plugins no workspace, or latency-critical serving loops in which
+ * a cudaMalloc (it may synchronize the device) is not allowed once serving
+ * has started.
+ *
+ * Scratch: one array of ZQ_NOALLOC_SCRATCH_BYTES in device memory, owned by
+ * the library.  Every GPU that loads the library holds it until the process
+ * exits.  A call needs round_up(4*T, 256) + 4*T*N bytes of it; a larger
+ * problem returns ZQ_ERR_SCRATCH before anything is enqueued.
+ * Set-up: the first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.
+ * Sharing: all calls on a device use the same array and it keeps the last
+ * call's contents (the call clears what must start at zero).  Calls whose
+ * GPU work overlaps -- on different streams, or from different threads --
+ * race on the array and give wrong results; order them on one stream.
+ * Arguments, layouts and the other errors as zq_w8a8_linear: y is int8
+ * [T, N], s_tok_out fp32 [T]; both outputs are required. */
+#define ZQ_NOALLOC_SCRATCH_BYTES (64u << 20)
+int zq_w8a8_linear_requant_noalloc(const int8_t* xq, const float* s_tok, int64_t T, int64_t K,
+                                   const int8_t* Wq, const float* s_grp, int64_t N,
+                                   int64_t group_rows, const float* bias, int act,
+                                   int8_t* y, float* s_tok_out, void* stream);
 
 /* ---- diagnostics ----------------------------------------------------------
  * zq_device_status: synchronizes `stream`, then reads and clears the device

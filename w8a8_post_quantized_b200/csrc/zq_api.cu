@@ -164,6 +164,7 @@ const char* zq_status_string(int status) {
         case ZQ_ERR_TIMEOUT: return "a bounded device-side wait expired";
         case ZQ_ERR_WORKSPACE: return "workspace missing or too small";
         case ZQ_ERR_DEVICE: return "current device is not an sm_100 (B200-class) GPU";
+        case ZQ_ERR_SCRATCH: return "problem exceeds the fixed scratch array of the no-allocation entry point";
         default: return "unknown status";
     }
 }

@@ -21,6 +21,8 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libzq.so")
 # ---- enums, mirroring include/zq.h ---------------------------------------
 ZQ_OK, ZQ_ERR_NULL, ZQ_ERR_SHAPE, ZQ_ERR_ALIGN, ZQ_ERR_OVERFLOW = 0, 1, 2, 3, 4
 ZQ_ERR_DTYPE, ZQ_ERR_CUDA, ZQ_ERR_TIMEOUT, ZQ_ERR_WORKSPACE, ZQ_ERR_DEVICE = 5, 6, 7, 8, 9
+ZQ_ERR_SCRATCH = 10
+ZQ_NOALLOC_SCRATCH_BYTES = 64 << 20
 ZQ_F32, ZQ_BF16 = 0, 1
 ZQ_ACT_NONE, ZQ_ACT_GELU = 0, 1
 ZQ_OUT_F32, ZQ_OUT_BF16, ZQ_OUT_I8_REQUANT, ZQ_OUT_I32_RAW = 0, 1, 2, 3
@@ -31,6 +33,7 @@ EXPORTED = (
     "zq_quantize_weights", "zq_ln_quant", "zq_act_quant", "zq_w8a8_linear_workspace",
     "zq_w8a8_linear", "zq_linear_block_workspace", "zq_linear_block", "zq_device_status",
     "zq_status_string", "zq_last_cuda_error", "zq_version", "zq_launch_count",
+    "zq_w8a8_linear_requant_noalloc",
 )
 
 
@@ -69,6 +72,7 @@ def lib() -> ctypes.CDLL:
         "zq_last_cuda_error": (ctypes.c_char_p, []),
         "zq_version": (I, []),
         "zq_launch_count": (ctypes.c_uint64, []),
+        "zq_w8a8_linear_requant_noalloc": (I, [P, P, I64, I64, P, P, I64, I64, P, I, P, P, P]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -179,6 +183,23 @@ def zq_linear_block(x, gamma, beta, eps, Wq, s_grp, group_rows, bias=None, act=Z
                                  int(out_kind), _p(y), _p(s_tok_out), _p(workspace), ws_bytes,
                                  _s(stream)), "zq_linear_block")
     return (y, s_tok_out) if out_kind == ZQ_OUT_I8_REQUANT else y
+
+
+def zq_w8a8_linear_requant_noalloc(xq, s_tok, Wq, s_grp, group_rows, bias=None,
+                                   act=ZQ_ACT_GELU, y=None, s_tok_out=None, stream=None):
+    """Requantizing linear that uses the library's fixed scratch array instead of
+    a workspace (for callers that cannot allocate device memory).  The outputs
+    must be passed in by such callers; they are allocated here only as a
+    convenience for callers that can."""
+    T, K = xq.shape
+    N = Wq.shape[0]
+    y = torch.empty((T, N), dtype=torch.int8, device=xq.device) if y is None else y
+    s_tok_out = torch.empty(T, dtype=torch.float32, device=xq.device) if s_tok_out is None else s_tok_out
+    _check(lib().zq_w8a8_linear_requant_noalloc(_p(xq), _p(s_tok), T, K, _p(Wq), _p(s_grp), N,
+                                                group_rows, _p(bias), int(act), _p(y),
+                                                _p(s_tok_out), _s(stream)),
+           "zq_w8a8_linear_requant_noalloc")
+    return y, s_tok_out
 
 
 def zq_device_status(stream=None):
