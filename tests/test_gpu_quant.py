@@ -39,6 +39,10 @@ ROW_SHAPES = [
     (16, 64, "f32"), (1, 16, "bf16"), (7, 48, "bf16"), (33, 768, "bf16"), (129, 1024, "f32"),
     (5, 4096, "bf16"), (3, 6144, "bf16"), (2, 12288, "bf16"), (1, 65536, "bf16"),
     (300, 2064, "bf16"), (1000, 512, "f32"), (9, 12288, "f32"),
+    (3, 32768, "bf16"),      # longest row of the pipelined kernel (bf16)
+    (2, 40960, "bf16"),      # beyond it: the register kernel
+    (5, 16384, "f32"),       # longest fp32 row of the pipelined kernel
+    (4097, 768, "bf16"),     # partial last stage
 ]
 
 

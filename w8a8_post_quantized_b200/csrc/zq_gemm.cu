@@ -41,8 +41,9 @@ namespace {
 constexpr int BM = 128;         // MMA M: rows of the M-side operand per tile
 constexpr int BK = 128;         // K bytes per pipeline stage (one swizzle row)
 constexpr int UMMA_K = 32;      // K per tcgen05.mma of kind::i8
-constexpr int kThreads = 192;   // 6 warps
-constexpr int kEpiThreads = 128;
+// block = 2 warps (TMA producer, MMA issuer) + EW epilogue warps
+template <int EW>
+__host__ __device__ constexpr int block_threads() { return 64 + 32 * EW; }
 constexpr int A_STAGE = BM * BK;
 
 enum Epi { EPI_I32 = 0, EPI_F32 = 1, EPI_BF16 = 2, EPI_REQ = 3 };
@@ -71,21 +72,23 @@ struct Params {
 };
 
 template <int BN>
-constexpr uint32_t tmem_cols() {
+__host__ __device__ constexpr uint32_t tmem_cols() {
     return (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128 : (2 * BN <= 256) ? 256 : 512;
 }
 
 template <int BN, int STAGES>
-constexpr size_t smem_bytes() {
+__host__ __device__ constexpr size_t smem_bytes() {
     // 1024 alignment slack + operand ring + barriers/flags + epilogue staging
     return 1024 + (size_t)STAGES * (A_STAGE + BN * BK) + 256 + 2 * BN * sizeof(float);
 }
 
-template <int BN, int STAGES, bool SWAP, int EPI>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int BN, int STAGES, bool SWAP, int EPI, int EW>
+__global__ void __launch_bounds__(block_threads<EW>(), 1)
 w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const Params p) {
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128 is 16..256 step 16");
+    static_assert(EW % 4 == 0 && EW >= 4 && EW <= 16, "epilogue warps cover the 4 TMEM lane quarters");
+    constexpr int kEpiThreads = 32 * EW;
     constexpr int B_STAGE = BN * BK;
     constexpr int CW = (BN % 32 == 0) ? 32 : 16;  // epilogue column chunk
     constexpr uint32_t IDESC = idesc_i8(BM, BN);
@@ -119,7 +122,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar_tfull(b), 1);
-            mbar_init(bar_tempty(b), kEpiThreads / 32);
+            mbar_init(bar_tempty(b), EW);
         }
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
@@ -211,9 +214,15 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         __syncwarp();
     } else {
         // ------------------------------------------------ epilogue
+        // warp w may only read TMEM lanes 32*(w%4) .. +31; EW/4 warps share each
+        // lane quarter and split the tile's columns between them
+        constexpr int SLICES = EW / 4;
+        constexpr int CT = BN / CW;             // column chunks per tile
         const int quarter = warp & 3;           // TMEM lanes 32*quarter .. +31
+        const int slice = (warp - 2) >> 2;      // which share of the columns
+        const int c_begin = slice * CT / SLICES, c_end = (slice + 1) * CT / SLICES;
         const int r = quarter * 32 + lane;      // row of the tile this thread owns
-        const int et = threadIdx.x - 64;        // 0..127
+        const int et = threadIdx.x - 64;        // 0 .. 32*EW-1
         float* st_a = stage_f;                  // per-column scale (or token scale when swapped)
         float* st_b = stage_f + BN;             // per-column bias (non-swapped)
         uint32_t lt = 0;
@@ -255,7 +264,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             const uint32_t t_row = tmem_base + (uint32_t)(b * BN) + ((uint32_t)(quarter * 32) << 16);
 
 #pragma unroll 1
-            for (int c = 0; c < BN / CW; ++c) {
+            for (int c = c_begin; c < c_end; ++c) {
                 uint32_t v[CW];
                 if constexpr (CW == 32) tmem_ld_32x32b_x32(t_row + c * CW, v);
                 else tmem_ld_32x32b_x16(t_row + c * CW, v);
@@ -380,12 +389,12 @@ int make_tmap_i8(CUtensorMap* tm, const void* ptr, int64_t rows, int64_t K, int 
 
 constexpr int kMaxDevices = 64;
 
-template <int BN, int STAGES, bool SWAP, int EPI>
+template <int BN, int STAGES, bool SWAP, int EPI, int EW>
 int launch_cfg(const CUtensorMap& ta, const CUtensorMap& tb, const Params& p, const DeviceInfo& di,
                cudaStream_t st) {
     static_assert(smem_bytes<BN, STAGES>() <= 232448, "shared memory budget");
     static_assert(smem_bytes<BN, STAGES>() > 116 * 1024, "one CTA per SM (TMEM ownership)");
-    auto kern = w8a8_gemm_kernel<BN, STAGES, SWAP, EPI>;
+    auto kern = w8a8_gemm_kernel<BN, STAGES, SWAP, EPI, EW>;
     static bool attr_set[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -399,19 +408,42 @@ int launch_cfg(const CUtensorMap& ta, const CUtensorMap& tb, const Params& p, co
     const int tiles = ((p.M + BM - 1) / BM) * ((p.N + BN - 1) / BN);
     const int grid = tiles < di.sm_count ? tiles : di.sm_count;
     count_launch();
-    kern<<<grid, kThreads, smem_bytes<BN, STAGES>(), st>>>(ta, tb, p);
+    kern<<<grid, block_threads<EW>(), smem_bytes<BN, STAGES>(), st>>>(ta, tb, p);
     return cuda_status(cudaGetLastError());
 }
 
 template <int BN, int STAGES, bool SWAP>
 int launch_epi(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const Params& p,
                const DeviceInfo& di, cudaStream_t st) {
+    // the epilogue is the long pole for short K loops: 16 warps (4 per SM
+    // sub-partition) when it dequantizes, 8 for raw int32 and the decode shapes
+    constexpr int EW = SWAP ? 8 : 16;
     switch (epi) {
-        case EPI_I32: return launch_cfg<BN, STAGES, SWAP, EPI_I32>(ta, tb, p, di, st);
-        case EPI_F32: return launch_cfg<BN, STAGES, SWAP, EPI_F32>(ta, tb, p, di, st);
-        case EPI_BF16: return launch_cfg<BN, STAGES, SWAP, EPI_BF16>(ta, tb, p, di, st);
-        default: return launch_cfg<BN, STAGES, SWAP, EPI_REQ>(ta, tb, p, di, st);
+        case EPI_I32: return launch_cfg<BN, STAGES, SWAP, EPI_I32, 8>(ta, tb, p, di, st);
+        case EPI_F32: return launch_cfg<BN, STAGES, SWAP, EPI_F32, EW>(ta, tb, p, di, st);
+        case EPI_BF16: return launch_cfg<BN, STAGES, SWAP, EPI_BF16, EW>(ta, tb, p, di, st);
+        default: return launch_cfg<BN, STAGES, SWAP, EPI_REQ, EW>(ta, tb, p, di, st);
     }
+}
+
+// Tile width for the non-swapped kernel: every CTA runs whole tiles, so the
+// time goes as (waves of tiles) x (tile width); take the cheapest, wider on
+// ties (fewer A re-reads, less shared-memory traffic per MMA).
+int pick_bn(int64_t T, int64_t N, int sms) {
+    const int cands[3] = {256, 192, 128};
+    int best = 256;
+    int64_t best_cost = -1;
+    const int64_t m_tiles = (T + BM - 1) / BM;
+    for (int bn : cands) {
+        const int64_t tiles = m_tiles * ((N + bn - 1) / bn);
+        const int64_t waves = (tiles + sms - 1) / sms;
+        const int64_t cost = waves * bn;
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = bn;
+        }
+    }
+    return best;
 }
 
 }  // namespace
@@ -452,10 +484,11 @@ int launch_w8a8_gemm(const LinearArgs& a, const DeviceInfo& di, cudaStream_t st)
     }
     p.M = (int)a.T;
     p.N = (int)a.N;
-    const int bn = a.N >= 256 ? 256 : 128;
+    const int bn = pick_bn(a.T, a.N, di.sm_count);
     if ((rc = make_tmap_i8(&ta, a.xq, a.T, a.K, BM))) return rc;
     if ((rc = make_tmap_i8(&tb, a.Wq, a.N, a.K, bn))) return rc;
     if (bn == 256) return launch_epi<256, 4, false>(epi, ta, tb, p, di, st);
+    if (bn == 192) return launch_epi<192, 5, false>(epi, ta, tb, p, di, st);
     return launch_epi<128, 6, false>(epi, ta, tb, p, di, st);
 }
 

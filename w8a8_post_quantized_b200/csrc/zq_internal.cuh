@@ -130,6 +130,89 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint
         : "memory");
 }
 
+// 1-D bulk copy global -> shared (contiguous bytes), completion counted on
+// `bar`.  Addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+// Round to nearest even and saturate to [-128, 127] in one conversion.  For
+// |y| <= absmax and inv = fp32(127/absmax), |y*inv| <= 127*(1+2^-24), so the
+// result always lies in [-127, 127] and equals clamp(rint(y*inv), -127, 127).
+__device__ __forceinline__ uint32_t quant_code_sat(float y, float inv) {
+    uint32_t r;
+    asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(r) : "f"(__fmul_rn(y, inv)));
+    return r & 0xFFu;
+}
+
+// ------------------------------------------------- packed fp32 pairs (sm_100)
+// A pair of fp32 values in one 64-bit register; add/sub/mul/fma on the pair
+// issue as one instruction (each lane is still IEEE round-to-nearest).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
+// Codes of four fp32 values packed little-endian into one word.
+// t = fl(y * inv) as a packed multiply; then fl(t + 1.5*2^23) (a scalar add
+// with explicit round-to-nearest, which is never contracted with the multiply)
+// holds rint(t), ties to even, in its low mantissa bits; the low byte is the
+// two's-complement code.  For |y| <= absmax, |t| <= 127*(1+2^-24), so no clamp
+// is ever active and the code equals clamp(rint(fl(y*inv)), -127, 127).
+// (A packed add here would be fused with the packed multiply into one FMA,
+// rounding once instead of twice.)
+__device__ __forceinline__ uint32_t quant4_packed(uint64_t y01, uint64_t y23, uint64_t inv2) {
+    const float magic = 12582912.0f;  // 1.5 * 2^23
+    float t0, t1, t2, t3;
+    f2_unpack(f2_mul(y01, inv2), t0, t1);
+    f2_unpack(f2_mul(y23, inv2), t2, t3);
+    const uint32_t c0 = __float_as_uint(__fadd_rn(t0, magic));
+    const uint32_t c1 = __float_as_uint(__fadd_rn(t1, magic));
+    const uint32_t c2 = __float_as_uint(__fadd_rn(t2, magic));
+    const uint32_t c3 = __float_as_uint(__fadd_rn(t3, magic));
+    return __byte_perm(__byte_perm(c0, c1, 0x0040), __byte_perm(c2, c3, 0x0040), 0x5410);
+}
+
+// Codes of four values with a single rounding: rint(y*inv) computed as one
+// fused multiply-add with the 1.5*2^23 constant.  It differs from the
+// two-rounding form above only when y*inv lies within half an fp32 ulp of a
+// tie; used where y is itself an fp32 approximation (LayerNorm, GeLU) and the
+// codes are compared within a tolerance, never on the bit-exact paths.
+__device__ __forceinline__ uint32_t quant4_packed_fused(uint64_t y01, uint64_t y23, uint64_t inv2) {
+    const uint64_t magic = 0x4B4000004B400000ull;  // (1.5*2^23, 1.5*2^23)
+    const uint64_t m01 = f2_fma(y01, inv2, magic);
+    const uint64_t m23 = f2_fma(y23, inv2, magic);
+    return __byte_perm(__byte_perm((uint32_t)m01, (uint32_t)(m01 >> 32), 0x0040),
+                       __byte_perm((uint32_t)m23, (uint32_t)(m23 >> 32), 0x0040), 0x5410);
+}
+
 // ---------------------------------------------------------------- tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
@@ -265,6 +348,11 @@ int launch_ln_quant(const void* x, int x_dtype, int64_t T, int64_t H, const floa
                     cudaStream_t st);
 int launch_act_quant(const void* x, int x_dtype, int64_t T, int64_t H, const float* bias, int act,
                      int8_t* q, float* s_tok, const DeviceInfo& di, cudaStream_t st);
+// Pipelined row quantizers (bulk copies into a shared-memory ring); return
+// ZQ_ERR_SHAPE when H is outside their range so the caller can fall back.
+int launch_rowq_pipe(const void* x, int x_dtype, int64_t T, int64_t H, bool ln, const float* gamma,
+                     const float* beta, float eps, const float* bias, int act, int8_t* q,
+                     float* s_tok, const DeviceInfo& di, cudaStream_t st);
 int launch_requant_rows(const float* h, int64_t T, int64_t N, const uint32_t* amax_bits, int8_t* q,
                         float* s_tok, const DeviceInfo& di, cudaStream_t st);
 

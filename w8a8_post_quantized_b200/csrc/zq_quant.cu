@@ -124,7 +124,7 @@ __device__ __forceinline__ float row_max(float v, float* sbuf) {
 }
 
 template <int RT>
-constexpr int block_threads() { return RT >= 256 ? RT : 256; }
+__host__ __device__ constexpr int block_threads() { return RT >= 256 ? RT : 256; }
 
 // ------------------------------------------------- LayerNorm + quantize
 
@@ -381,15 +381,20 @@ static int launch_act_typed(const Tin* x, int64_t T, int64_t H, const float* bia
 }  // namespace
 
 int launch_ln_quant(const void* x, int x_dtype, int64_t T, int64_t H, const float* gamma,
-                    const float* beta, float eps, int8_t* q, float* s_tok, const DeviceInfo&,
+                    const float* beta, float eps, int8_t* q, float* s_tok, const DeviceInfo& di,
                     cudaStream_t st) {
+    // pipelined kernel first; rows too long for it use the register kernel below
+    const int rc = launch_rowq_pipe(x, x_dtype, T, H, true, gamma, beta, eps, nullptr, 0, q, s_tok, di, st);
+    if (rc != ZQ_ERR_SHAPE) return rc;
     if (x_dtype == ZQ_BF16)
         return launch_ln_typed(static_cast<const uint16_t*>(x), T, H, gamma, beta, eps, q, s_tok, st);
     return launch_ln_typed(static_cast<const float*>(x), T, H, gamma, beta, eps, q, s_tok, st);
 }
 
 int launch_act_quant(const void* x, int x_dtype, int64_t T, int64_t H, const float* bias, int act,
-                     int8_t* q, float* s_tok, const DeviceInfo&, cudaStream_t st) {
+                     int8_t* q, float* s_tok, const DeviceInfo& di, cudaStream_t st) {
+    const int rc = launch_rowq_pipe(x, x_dtype, T, H, false, nullptr, nullptr, 0.f, bias, act, q, s_tok, di, st);
+    if (rc != ZQ_ERR_SHAPE) return rc;
     if (x_dtype == ZQ_BF16)
         return launch_act_typed(static_cast<const uint16_t*>(x), T, H, bias, act, q, s_tok, st);
     return launch_act_typed(static_cast<const float*>(x), T, H, bias, act, q, s_tok, st);

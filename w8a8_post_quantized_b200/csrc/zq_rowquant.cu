@@ -1,0 +1,475 @@
+// zq_rowquant.cu -- pipelined per-token quantizers for sm_100a:
+// fused LayerNorm + quantize and fused (bias +) GeLU + quantize.
+//
+// Sources: "[2022 NeurIPS] ZeroQuant: Efficient and Affordable Post-Training
+// Quantization for Large-Scale Transformers" (token-wise quantization fused
+// with the preceding element-wise or reduction op: "LN/GeLU + Quantize") and
+// "探秘Transformer系列之（36）— 大模型量化方案" §1.1.2 (absmax rule into
+// [-127, 127]) and §1.2.2 (one dynamic scale per token, computed at run
+// time, the quantizer fused with LayerNorm).
+//
+// HBM-bound: each input byte is read once and each code written once.  A
+// persistent CTA streams blocks of R consecutive rows (contiguous in memory)
+// into a ring of shared-memory stages with one 1-D bulk async copy per stage,
+// so several stages per SM are in flight while the current one is processed.
+// Rows are processed by teams of TPR threads (a warp for short rows, the whole
+// CTA for long ones); each thread holds PPT pieces of the row in registers (a
+// piece is 16 input bytes: 8 bf16 or 4 fp32 values, read from shared memory
+// without bank conflicts), so the statistics need no second pass over memory.
+#include "zq_internal.cuh"
+
+namespace zq {
+namespace {
+
+constexpr int kSiteRowqFull = 0x401;
+constexpr int kRingBytes = 192 * 1024;      // shared-memory ring budget per CTA
+constexpr int kStageTarget = 24 * 1024;     // preferred bytes per stage
+constexpr int kMaxStages = 8;
+constexpr int kRingOffset = 1024;           // barriers + reduction slots before the ring
+
+// A piece is 16 input bytes held as NP packed fp32 pairs.
+template <typename Tin>
+struct Piece;
+
+template <>
+struct Piece<uint16_t> {  // bf16 bit patterns: 8 values, 4 pairs
+    static constexpr int EPP = 8;
+    static constexpr int NP = 4;
+    static __device__ __forceinline__ void load(const uint16_t* p, uint64_t (&v)[NP]) {
+        const uint4 a = *reinterpret_cast<const uint4*>(p);
+        v[0] = f2_pack(bf16_lo(a.x), bf16_hi(a.x));
+        v[1] = f2_pack(bf16_lo(a.y), bf16_hi(a.y));
+        v[2] = f2_pack(bf16_lo(a.z), bf16_hi(a.z));
+        v[3] = f2_pack(bf16_lo(a.w), bf16_hi(a.w));
+    }
+};
+
+template <>
+struct Piece<float> {  // 4 values, 2 pairs
+    static constexpr int EPP = 4;
+    static constexpr int NP = 2;
+    static __device__ __forceinline__ void load(const float* p, uint64_t (&v)[NP]) {
+        const ulonglong2 a = *reinterpret_cast<const ulonglong2*>(p);
+        v[0] = a.x;
+        v[1] = a.y;
+    }
+};
+
+// NP pairs of fp32 parameters (gamma, beta or bias) of piece p.  A piece's
+// parameters are NP/2 16-byte quarters.  In global memory they are
+// contiguous; the shared-memory copy stores quarter h of every piece together
+// (index h*nP + p), so the 16-byte loads of consecutive threads are
+// contiguous and free of bank conflicts.
+template <int NP, bool SMEM>
+__device__ __forceinline__ void load_param_pairs(const float* base, int p, int nP, uint64_t (&v)[NP]) {
+#pragma unroll
+    for (int h = 0; h < NP / 2; ++h) {
+        const ulonglong2* src =
+            reinterpret_cast<const ulonglong2*>(SMEM ? base + ((size_t)h * nP + p) * 4 : base + (size_t)p * 2 * NP + h * 4);
+        const ulonglong2 a = SMEM ? *src : __ldg(src);
+        v[2 * h] = a.x;
+        v[2 * h + 1] = a.y;
+    }
+}
+
+__device__ __forceinline__ float f2_hsum(uint64_t v) {
+    float a, b;
+    f2_unpack(v, a, b);
+    return a + b;
+}
+
+__device__ __forceinline__ float f2_absmax(float m, uint64_t v) {
+    float a, b;
+    f2_unpack(v, a, b);
+    return fmaxf(m, fmaxf(fabsf(a), fabsf(b)));
+}
+
+// FUSED: single-rounding codes (LayerNorm / GeLU paths, see quant4_packed_fused).
+template <int NP, bool FUSED>
+__device__ __forceinline__ void store_piece_codes(int8_t* dst, const uint64_t (&y)[NP], uint64_t inv2) {
+    if constexpr (NP == 4) {
+        uint2 o;
+        o.x = FUSED ? quant4_packed_fused(y[0], y[1], inv2) : quant4_packed(y[0], y[1], inv2);
+        o.y = FUSED ? quant4_packed_fused(y[2], y[3], inv2) : quant4_packed(y[2], y[3], inv2);
+        __stcs(reinterpret_cast<uint2*>(dst), o);
+    } else {
+        __stcs(reinterpret_cast<uint32_t*>(dst),
+               FUSED ? quant4_packed_fused(y[0], y[1], inv2) : quant4_packed(y[0], y[1], inv2));
+    }
+}
+
+// Reductions over the TPR threads of one team.  Teams smaller than the CTA
+// use their own named barrier (id 1 + team) and their own reduction slots.
+template <int TPR, int BLOCK>
+struct Team {
+    static __device__ __forceinline__ void sync(int team) {
+        if constexpr (TPR == BLOCK) __syncthreads();
+        else named_bar_sync(1 + team, TPR);
+    }
+    // xor-shuffle offsets stay inside a team when TPR < 32 (two teams per warp)
+    static constexpr int kTopLane = TPR < 32 ? TPR / 2 : 16;
+    static __device__ __forceinline__ float sum(float v, float* red, int team) {
+#pragma unroll
+        for (int o = kTopLane; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+        if constexpr (TPR <= 32) {
+            return v;
+        } else {
+            constexpr int W = TPR / 32;
+            float* slot = red + team * W;
+            if ((threadIdx.x & 31) == 0) slot[(threadIdx.x % TPR) >> 5] = v;
+            sync(team);
+            float t = 0.0f;
+#pragma unroll
+            for (int i = 0; i < W; ++i) t += slot[i];
+            sync(team);
+            return t;
+        }
+    }
+    // Merge per-thread (count, mean, sum of squared deviations) over the team
+    // with Chan's pairwise update; returns the team's mean and M2.
+    static __device__ __forceinline__ void stats(float n, float mean, float m2, float* red, int team,
+                                                 float& mean_out, float& m2_out) {
+#pragma unroll
+        for (int o = kTopLane; o > 0; o >>= 1) {
+            const float nb = __shfl_xor_sync(0xFFFFFFFFu, n, o);
+            const float mb = __shfl_xor_sync(0xFFFFFFFFu, mean, o);
+            const float qb = __shfl_xor_sync(0xFFFFFFFFu, m2, o);
+            merge(n, mean, m2, nb, mb, qb);
+        }
+        if constexpr (TPR > 32) {
+            constexpr int W = TPR / 32;
+            float* slot = red + team * W * 3;
+            const int w = (threadIdx.x % TPR) >> 5;
+            if ((threadIdx.x & 31) == 0) {
+                slot[3 * w] = n;
+                slot[3 * w + 1] = mean;
+                slot[3 * w + 2] = m2;
+            }
+            sync(team);
+            n = slot[0];
+            mean = slot[1];
+            m2 = slot[2];
+#pragma unroll
+            for (int i = 1; i < W; ++i) merge(n, mean, m2, slot[3 * i], slot[3 * i + 1], slot[3 * i + 2]);
+            sync(team);
+        }
+        mean_out = mean;
+        m2_out = m2;
+    }
+    static __device__ __forceinline__ void merge(float& n, float& mean, float& m2, float nb, float mb,
+                                                 float qb) {
+        const float nt = n + nb;
+        if (nt > 0.0f) {
+            const float d = mb - mean;
+            const float f = __fdividef(nb, nt);
+            mean = fmaf(d, f, mean);
+            m2 = m2 + qb + d * d * n * f;
+            n = nt;
+        }
+    }
+    static __device__ __forceinline__ float max(float v, float* red, int team) {
+#pragma unroll
+        for (int o = kTopLane; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+        if constexpr (TPR <= 32) {
+            return v;
+        } else {
+            constexpr int W = TPR / 32;
+            float* slot = red + team * W;
+            if ((threadIdx.x & 31) == 0) slot[(threadIdx.x % TPR) >> 5] = v;
+            sync(team);
+            float t = 0.0f;
+#pragma unroll
+            for (int i = 0; i < W; ++i) t = fmaxf(t, slot[i]);
+            sync(team);
+            return t;
+        }
+    }
+};
+
+template <typename Tin, bool LN, int TPR, int PPT, int BLOCK, bool SMEMP>
+__global__ void __launch_bounds__(BLOCK, 1)
+rowq_pipe_kernel(const Tin* __restrict__ x, int T, int H, float inv_h, int R, int nstages,
+                 const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
+                 const float* __restrict__ bias, int act, int8_t* __restrict__ q,
+                 float* __restrict__ s_tok, int* status) {
+    constexpr int EPP = Piece<Tin>::EPP;
+    constexpr int NP = Piece<Tin>::NP;
+    constexpr int TEAMS = BLOCK / TPR;
+    using TM = Team<TPR, BLOCK>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const uint32_t bar0 = smem_u32(smem);
+    float* red = reinterpret_cast<float*>(smem + 128);
+    // per-column parameters (gamma and beta, or bias) copied once per CTA
+    const int n_par = LN ? 2 : (bias ? 1 : 0);
+    float* spar = reinterpret_cast<float*>(smem + kRingOffset);
+    uint8_t* ring = smem + kRingOffset + (SMEMP ? (size_t)n_par * H * sizeof(float) : 0);
+    const int row_bytes = H * (int)sizeof(Tin);
+    const int stage_bytes = R * row_bytes;
+    const int nP = H / EPP;
+    const int team = threadIdx.x / TPR;
+    const int tt = threadIdx.x % TPR;
+    const int n_units = (T + R - 1) / R;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < nstages; ++s) mbar_init(bar0 + 8u * s, 1);
+        fence_proxy_async_smem();
+        fence_barrier_init();
+    }
+    if constexpr (SMEMP) {
+        const float* src0 = LN ? gamma : bias;
+        constexpr int QPP = NP / 2;  // 16-byte quarters per piece
+        for (int i = threadIdx.x; i < H / 4; i += BLOCK) {
+            const int dst = (i % QPP) * nP + i / QPP;
+            if (n_par >= 1) reinterpret_cast<float4*>(spar)[dst] = __ldg(reinterpret_cast<const float4*>(src0) + i);
+            if (n_par == 2) reinterpret_cast<float4*>(spar + H)[dst] = __ldg(reinterpret_cast<const float4*>(beta) + i);
+        }
+    }
+    const float* pg = SMEMP ? spar : gamma;
+    const float* pb = SMEMP ? spar + H : beta;
+    const float* pbias = SMEMP ? spar : bias;
+    __syncthreads();
+
+    auto issue = [&](int u, int s) {
+        const int rows = min(R, T - u * R);
+        const uint32_t bytes = (uint32_t)(rows * row_bytes);
+        mbar_arrive_expect_tx(bar0 + 8u * s, bytes);
+        bulk_load(smem_u32(ring + (size_t)s * stage_bytes), x + (int64_t)u * R * H, bytes, bar0 + 8u * s);
+    };
+    if (threadIdx.x == 0)
+        for (int j = 0; j < nstages; ++j) {
+            const int u = blockIdx.x + j * gridDim.x;
+            if (u < n_units) issue(u, j);
+        }
+
+    int j = 0;
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++j) {
+        const int s = j % nstages;
+        const uint32_t ph = (uint32_t)(j / nstages) & 1u;
+        const bool ok = mbar_wait(bar0 + 8u * s, ph, nullptr, status, kSiteRowqFull);
+        if (!__syncthreads_and(ok)) {
+            // a copy never landed: wait (bounded) for the others in flight, then stop
+            if (threadIdx.x == 0)
+                for (int k = 1; k < nstages; ++k) {
+                    const int jj = j + k;
+                    if (blockIdx.x + jj * gridDim.x < n_units)
+                        mbar_wait(bar0 + 8u * (jj % nstages), (uint32_t)(jj / nstages) & 1u, nullptr,
+                                  status, kSiteRowqFull);
+                }
+            break;
+        }
+        const int rows = min(R, T - u * R);
+        const Tin* sx = reinterpret_cast<const Tin*>(ring + (size_t)s * stage_bytes);
+        // all teams sharing a warp run the same number of iterations (their
+        // shuffles use the full warp); a team past the last row works on a
+        // masked row and stores nothing
+        constexpr int TPW = TPR < 32 ? 32 / TPR : 1;
+        for (int rb = team - team % TPW; rb < rows; rb += TEAMS) {
+            const int r = rb + team % TPW;
+            const bool row_ok = r < rows;
+            const Tin* xr = sx + (size_t)(row_ok ? r : 0) * H;
+            const int64_t row = (int64_t)u * R + r;
+            uint64_t v[PPT][NP];
+            bool okp[PPT];
+#pragma unroll
+            for (int k = 0; k < PPT; ++k) {
+                const int p = k * TPR + tt;
+                okp[k] = row_ok && p < nP;
+                if (okp[k]) Piece<Tin>::load(xr + p * EPP, v[k]);
+                else {
+#pragma unroll
+                    for (int i = 0; i < NP; ++i) v[k][i] = 0ull;
+                }
+            }
+            float amax = 0.0f;
+            if constexpr (LN) {
+                // per-thread mean and squared deviations (two passes over the
+                // registers, four independent accumulators each), merged over
+                // the team in one Chan reduction
+                uint64_t sa[4] = {0ull, 0ull, 0ull, 0ull};
+                int nv = 0;
+#pragma unroll
+                for (int k = 0; k < PPT; ++k) {
+                    nv += okp[k] ? EPP : 0;
+#pragma unroll
+                    for (int i = 0; i < NP; ++i) sa[(k * NP + i) & 3] = f2_add(sa[(k * NP + i) & 3], v[k][i]);
+                }
+                const float n_loc = (float)nv;
+                const float mean_loc =
+                    nv ? f2_hsum(f2_add(f2_add(sa[0], sa[1]), f2_add(sa[2], sa[3]))) * __frcp_rn(n_loc) : 0.0f;
+                const uint64_t ml2 = f2_pack(mean_loc, mean_loc);
+                uint64_t da[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+                for (int k = 0; k < PPT; ++k)
+                    if (okp[k]) {
+#pragma unroll
+                        for (int i = 0; i < NP; ++i) {
+                            const uint64_t d = f2_sub(v[k][i], ml2);
+                            da[(k * NP + i) & 3] = f2_fma(d, d, da[(k * NP + i) & 3]);
+                        }
+                    }
+                float mean, m2;
+                TM::stats(n_loc, mean_loc, f2_hsum(f2_add(f2_add(da[0], da[1]), f2_add(da[2], da[3]))),
+                          red, team, mean, m2);
+                const float rstd = rsqrtf(fmaf(m2, inv_h, eps));
+                const uint64_t mean2 = f2_pack(mean, mean);
+                const uint64_t rstd2 = f2_pack(rstd, rstd);
+                float am[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+                for (int k = 0; k < PPT; ++k)
+                    if (okp[k]) {
+                        const int p = k * TPR + tt;
+                        uint64_t g[NP], b[NP];
+                        load_param_pairs<NP, SMEMP>(pg, p, nP, g);
+                        load_param_pairs<NP, SMEMP>(pb, p, nP, b);
+#pragma unroll
+                        for (int i = 0; i < NP; ++i) {
+                            const uint64_t a = f2_mul(rstd2, g[i]);
+                            const uint64_t y = f2_fma(f2_sub(v[k][i], mean2), a, b[i]);
+                            v[k][i] = y;
+                            am[(k * NP + i) & 3] = f2_absmax(am[(k * NP + i) & 3], y);
+                        }
+                    }
+                amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
+            } else {
+                float am[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+                for (int k = 0; k < PPT; ++k)
+                    if (okp[k]) {
+                        if (bias) {
+                            uint64_t b[NP];
+                            load_param_pairs<NP, SMEMP>(pbias, k * TPR + tt, nP, b);
+#pragma unroll
+                            for (int i = 0; i < NP; ++i) v[k][i] = f2_add(v[k][i], b[i]);
+                        }
+                        if (act == ZQ_ACT_GELU) {
+#pragma unroll
+                            for (int i = 0; i < NP; ++i) {
+                                float lo, hi;
+                                f2_unpack(v[k][i], lo, hi);
+                                v[k][i] = f2_pack(gelu_f(lo), gelu_f(hi));
+                            }
+                        }
+#pragma unroll
+                        for (int i = 0; i < NP; ++i) am[(k * NP + i) & 3] = f2_absmax(am[(k * NP + i) & 3], v[k][i]);
+                    }
+                amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
+            }
+            amax = TM::max(amax, red, team);
+            float scale, inv;
+            absmax_scales(amax, scale, inv);
+            const uint64_t inv2 = f2_pack(inv, inv);
+            int8_t* qr = q + row * H;
+            if (LN || act == ZQ_ACT_GELU) {
+#pragma unroll
+                for (int k = 0; k < PPT; ++k)
+                    if (okp[k]) store_piece_codes<NP, true>(qr + (k * TPR + tt) * EPP, v[k], inv2);
+            } else {
+#pragma unroll
+                for (int k = 0; k < PPT; ++k)
+                    if (okp[k]) store_piece_codes<NP, false>(qr + (k * TPR + tt) * EPP, v[k], inv2);
+            }
+            if (row_ok && tt == 0) s_tok[row] = scale;
+        }
+        __syncthreads();  // every team is done with stage s
+        if (threadIdx.x == 0) {
+            const int u2 = u + nstages * gridDim.x;
+            if (u2 < n_units) issue(u2, s);
+        }
+    }
+}
+
+template <typename Tin, bool LN>
+using PipeKernel = void (*)(const Tin*, int, int, float, int, int, const float*, const float*, float,
+                            const float*, int, int8_t*, float*, int*);
+
+// (TPR, PPT, BLOCK) shapes: a team of TPR threads covers TPR*PPT pieces.
+struct Shape {
+    int tpr, ppt, block;
+};
+// Each thread holds 6-8 pieces (48-64 values) so the per-row costs
+// (reductions, divisions) are spread over many elements, with 16 warps per SM.
+// Teams are half a warp for short rows (two rows per warp, no barriers), one
+// or more warps for longer rows.
+constexpr Shape kShapes[] = {{16, 1, 512},   {16, 2, 512},  {16, 4, 512},  {16, 6, 512},
+                             {16, 8, 512},   {32, 8, 512},  {64, 8, 512},  {128, 6, 512},
+                             {128, 8, 512},  {256, 6, 512}, {256, 8, 512}, {256, 16, 256}};
+constexpr int kNumShapes = 12;
+constexpr int kFirstGlobalParamShape = 10;  // from here on parameters stay in global memory
+
+template <typename Tin, bool LN>
+PipeKernel<Tin, LN> pipe_kernel(int idx) {
+    switch (idx) {
+        case 0: return rowq_pipe_kernel<Tin, LN, 16, 1, 512, true>;
+        case 1: return rowq_pipe_kernel<Tin, LN, 16, 2, 512, true>;
+        case 2: return rowq_pipe_kernel<Tin, LN, 16, 4, 512, true>;
+        case 3: return rowq_pipe_kernel<Tin, LN, 16, 6, 512, true>;
+        case 4: return rowq_pipe_kernel<Tin, LN, 16, 8, 512, true>;
+        case 5: return rowq_pipe_kernel<Tin, LN, 32, 8, 512, true>;
+        case 6: return rowq_pipe_kernel<Tin, LN, 64, 8, 512, true>;
+        case 7: return rowq_pipe_kernel<Tin, LN, 128, 6, 512, true>;
+        case 8: return rowq_pipe_kernel<Tin, LN, 128, 8, 512, true>;
+        case 9: return rowq_pipe_kernel<Tin, LN, 256, 6, 512, true>;
+        case 10: return rowq_pipe_kernel<Tin, LN, 256, 8, 512, false>;
+        default: return rowq_pipe_kernel<Tin, LN, 256, 16, 256, false>;
+    }
+}
+
+// Smallest shape whose team covers the row's pieces.
+int pick_shape(int pieces) {
+    for (int i = 0; i < kNumShapes; ++i)
+        if (kShapes[i].tpr * kShapes[i].ppt >= pieces) return i;
+    return -1;
+}
+
+template <typename Tin, bool LN>
+int launch_typed(const Tin* x, int64_t T, int64_t H, const float* gamma, const float* beta, float eps,
+                 const float* bias, int act, int8_t* q, float* s_tok, const DeviceInfo& di,
+                 cudaStream_t st) {
+    constexpr int EPP = Piece<Tin>::EPP;
+    const int idx = pick_shape((int)(H / EPP));
+    if (idx < 0 || T > (1ll << 30)) return ZQ_ERR_SHAPE;
+    const Shape sh = kShapes[idx];
+    const int teams = sh.block / sh.tpr;
+    const int row_bytes = (int)(H * sizeof(Tin));
+    // rows per stage: about kStageTarget bytes, a multiple of the team count;
+    // fewer rows per stage when the problem is too small to give every SM
+    // a few stages of work (idle teams are fine then)
+    int R = kStageTarget / row_bytes;
+    R = R < teams ? teams : R - R % teams;
+    const int64_t want_units = 2 * (int64_t)di.sm_count;
+    while (R > 1 && (T + R - 1) / R < want_units) R = R > teams ? R - teams : R / 2;
+    if (R < 1) R = 1;
+    const int stage_bytes = R * row_bytes;
+    const int n_par = LN ? 2 : (bias ? 1 : 0);
+    const size_t par_bytes = idx < kFirstGlobalParamShape ? (size_t)n_par * H * sizeof(float) : 0;
+    int nstages = (int)((kRingBytes - par_bytes) / stage_bytes);
+    if (nstages > kMaxStages) nstages = kMaxStages;
+    if (nstages < 2) return ZQ_ERR_SHAPE;
+    const int64_t n_units = (T + R - 1) / R;
+    const int grid = (int)(n_units < di.sm_count ? n_units : di.sm_count);
+    const size_t smem = kRingOffset + par_bytes + (size_t)nstages * stage_bytes;
+    auto kern = pipe_kernel<Tin, LN>(idx);
+    int rc = cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    if (rc) return rc;
+    count_launch();
+    kern<<<grid, sh.block, smem, st>>>(x, (int)T, (int)H, 1.0f / (float)H, R, nstages, gamma, beta,
+                                       eps, bias, act, q, s_tok, di.status_word);
+    return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
+int launch_rowq_pipe(const void* x, int x_dtype, int64_t T, int64_t H, bool ln, const float* gamma,
+                     const float* beta, float eps, const float* bias, int act, int8_t* q,
+                     float* s_tok, const DeviceInfo& di, cudaStream_t st) {
+    if (x_dtype == ZQ_BF16) {
+        const uint16_t* xb = static_cast<const uint16_t*>(x);
+        return ln ? launch_typed<uint16_t, true>(xb, T, H, gamma, beta, eps, nullptr, 0, q, s_tok, di, st)
+                  : launch_typed<uint16_t, false>(xb, T, H, nullptr, nullptr, 0.f, bias, act, q, s_tok, di, st);
+    }
+    const float* xf = static_cast<const float*>(x);
+    return ln ? launch_typed<float, true>(xf, T, H, gamma, beta, eps, nullptr, 0, q, s_tok, di, st)
+              : launch_typed<float, false>(xf, T, H, nullptr, nullptr, 0.f, bias, act, q, s_tok, di, st);
+}
+
+}  // namespace zq
