@@ -132,8 +132,13 @@ int run_linear(const int8_t* xq, const float* s_tok, int64_t T, int64_t K, const
     a.act = act;
     a.out_kind = out_kind;
     a.y = y;
+    a.s_tok_out = s_tok_out;
     int rc;
     if (out_kind == ZQ_OUT_I8_REQUANT) {
+        // fused: the row absmax is exchanged inside a thread-block cluster
+        rc = launch_w8a8_requant_cluster(a, di, st);
+        if (rc != ZQ_ERR_SHAPE) return rc;
+        // otherwise: fp32 epilogue output + row absmax in the workspace, then requantize
         uint8_t* w = static_cast<uint8_t*>(ws);
         a.h_ws = reinterpret_cast<float*>(w);
         a.amax_ws = reinterpret_cast<uint32_t*>(w + round_up((size_t)T * N * sizeof(float), kWsAlign));

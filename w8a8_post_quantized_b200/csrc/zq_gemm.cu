@@ -76,16 +76,24 @@ __host__ __device__ constexpr uint32_t tmem_cols() {
     return (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128 : (2 * BN <= 256) ? 256 : 512;
 }
 
-template <int BN, int STAGES>
+// Bytes of one 32x32 output box row: int32/fp32 outputs 128, bf16 64.
+template <int EPI>
+__host__ __device__ constexpr int out_row_bytes() { return EPI == EPI_BF16 ? 64 : 128; }
+
+template <int BN, int STAGES, bool SWAP, int EPI, int EW>
 __host__ __device__ constexpr size_t smem_bytes() {
-    // 1024 alignment slack + operand ring + barriers/flags + epilogue staging
-    return 1024 + (size_t)STAGES * (A_STAGE + BN * BK) + 256 + 2 * BN * sizeof(float);
+    // 1024 alignment slack + operand ring + output staging (one 32x32 box per
+    // epilogue warp, non-swapped only) + barriers/flags + per-column factors
+    // (bf16 outputs stage only the per-column scale; their bias is read
+    // through L1, which leaves room for a fourth pipeline stage at BN = 256)
+    return 1024 + (size_t)STAGES * (A_STAGE + BN * BK) + (SWAP ? 0 : (size_t)EW * 32 * out_row_bytes<EPI>()) +
+           256 + (EPI == EPI_I32 ? 0 : EPI == EPI_BF16 && !SWAP ? 1 : 2) * BN * sizeof(float);
 }
 
 template <int BN, int STAGES, bool SWAP, int EPI, int EW>
 __global__ void __launch_bounds__(block_threads<EW>(), 1)
 w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const Params p) {
+                 const __grid_constant__ CUtensorMap tmY, const Params p) {
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128 is 16..256 step 16");
     static_assert(EW % 4 == 0 && EW >= 4 && EW <= 16, "epilogue warps cover the 4 TMEM lane quarters");
     constexpr int kEpiThreads = 32 * EW;
@@ -98,9 +106,12 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* gbase = smem_raw + (base - raw);
+    constexpr int RB = out_row_bytes<EPI>();
+    constexpr uint32_t STG_BYTES = SWAP ? 0u : (uint32_t)EW * 32u * RB;
     const uint32_t sA = base;
     const uint32_t sB = base + STAGES * A_STAGE;
-    const uint32_t sBar = sB + STAGES * B_STAGE;
+    const uint32_t sStg = sB + STAGES * B_STAGE;  // 1024-aligned: every stage is a multiple of 1024
+    const uint32_t sBar = sStg + STG_BYTES;
     uint8_t* gBar = gbase + (sBar - base);
     // barrier layout: full[S], empty[S], tfull[2], tempty[2], drain
     auto bar_full = [&](int s) { return sBar + 8u * s; };
@@ -132,6 +143,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        if (!SWAP) tma_prefetch_desc(&tmY);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
@@ -223,6 +235,10 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const int c_begin = slice * CT / SLICES, c_end = (slice + 1) * CT / SLICES;
         const int r = quarter * 32 + lane;      // row of the tile this thread owns
         const int et = threadIdx.x - 64;        // 0 .. 32*EW-1
+        uint8_t* stg = gbase + (sStg - base) + (uint32_t)(warp - 2) * 32u * RB;  // this warp's box
+        const uint32_t stg_s = smem_u32(stg);
+        (void)stg;
+        (void)stg_s;
         float* st_a = stage_f;                  // per-column scale (or token scale when swapped)
         float* st_b = stage_f + BN;             // per-column bias (non-swapped)
         uint32_t lt = 0;
@@ -232,14 +248,15 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             const uint32_t tph = (lt >> 1) & 1u;
             // stage the per-column factors of this tile (previous readers done)
             named_bar_sync(1, kEpiThreads);
-            for (int i = et; i < BN; i += kEpiThreads) {
+            for (int i = et; EPI != EPI_I32 && i < BN; i += kEpiThreads) {
                 const int n = nt * BN + i;
                 const bool in = n < p.N;
                 if constexpr (SWAP) {
                     st_a[i] = (EPI != EPI_I32 && in) ? __ldg(p.s_tok + n) : 0.0f;
                 } else {
                     st_a[i] = (EPI != EPI_I32 && in) ? __ldg(p.s_grp + n / p.G) : 0.0f;
-                    st_b[i] = (EPI != EPI_I32 && in && p.bias) ? __ldg(p.bias + n) : 0.0f;
+                    if constexpr (EPI != EPI_BF16)
+                        st_b[i] = (EPI != EPI_I32 && in && p.bias) ? __ldg(p.bias + n) : 0.0f;
                 }
             }
             named_bar_sync(1, kEpiThreads);
@@ -262,6 +279,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             }
             float amax = 0.0f;
             const uint32_t t_row = tmem_base + (uint32_t)(b * BN) + ((uint32_t)(quarter * 32) << 16);
+            static_assert(SWAP || CW == 32, "non-swapped tiles are whole 32-column chunks");
 
 #pragma unroll 1
             for (int c = c_begin; c < c_end; ++c) {
@@ -271,48 +289,64 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 tmem_ld_wait();
                 const int n0 = nt * BN + c * CW;   // first N-side index of the chunk
                 if constexpr (!SWAP) {
-                    // thread owns token gm, columns n0 .. n0+CW-1 (output features)
-                    if (!row_ok) continue;
+                    // thread owns token gm (box row `lane`), columns n0 .. n0+31; the
+                    // warp's 32x32 box goes through shared memory to one TMA store
+                    // (rows >= M and columns >= N are clipped by the store)
+                    uint32_t w[RB / 4];
+                    if constexpr (EPI == EPI_I32) {
 #pragma unroll
-                    for (int h = 0; h < CW / 16; ++h) {
-                        const int nb = n0 + 16 * h;
-                        if (nb >= p.N) break;      // N % 16 == 0: 16-column groups are whole
-                        const int64_t off = (int64_t)gm * p.ldy + nb;
-                        if constexpr (EPI == EPI_I32) {
-                            int4* dst = reinterpret_cast<int4*>(static_cast<int32_t*>(p.y) + off);
+                        for (int j = 0; j < 32; ++j) w[j] = v[j];
+                    } else {
+                        float yv[32];
+                        // bf16 outputs read this chunk's bias through L1 (zero past N
+                        // or without bias); the others use the staged copy
+                        const bool has_b = EPI == EPI_BF16 && p.bias != nullptr && n0 < p.N;
+                        const float4* b4 = reinterpret_cast<const float4*>(p.bias + (has_b ? n0 : 0));
 #pragma unroll
-                            for (int q4 = 0; q4 < 4; ++q4)
-                                dst[q4] = make_int4((int)v[16 * h + 4 * q4], (int)v[16 * h + 4 * q4 + 1],
-                                                    (int)v[16 * h + 4 * q4 + 2], (int)v[16 * h + 4 * q4 + 3]);
-                        } else {
-                            float yv[16];
+                        for (int q = 0; q < 8; ++q) {
+                            float be[4];
+                            if constexpr (EPI == EPI_BF16) {
+                                const float4 t4 = (has_b && n0 + 4 * q < p.N) ? __ldg(b4 + q)
+                                                                               : make_float4(0.f, 0.f, 0.f, 0.f);
+                                be[0] = t4.x;
+                                be[1] = t4.y;
+                                be[2] = t4.z;
+                                be[3] = t4.w;
+                            } else {
 #pragma unroll
-                            for (int j = 0; j < 16; ++j) {
-                                const int i = c * CW + 16 * h + j;
-                                float t = fmaf(row_scale * st_a[i], (float)(int)v[16 * h + j], st_b[i]);
+                                for (int e = 0; e < 4; ++e) be[e] = st_b[c * CW + 4 * q + e];
+                            }
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int j = 4 * q + e;
+                                float t = fmaf(row_scale * st_a[c * CW + j], (float)(int)v[j], be[e]);
                                 if (p.act == ZQ_ACT_GELU) t = gelu_f(t);
                                 yv[j] = t;
                             }
-                            if constexpr (EPI == EPI_BF16) {
-                                uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.y) + off);
+                        }
+                        if constexpr (EPI == EPI_BF16) {
 #pragma unroll
-                                for (int q8 = 0; q8 < 2; ++q8)
-                                    dst[q8] = make_uint4(pack_bf16x2(yv[8 * q8 + 0], yv[8 * q8 + 1]),
-                                                         pack_bf16x2(yv[8 * q8 + 2], yv[8 * q8 + 3]),
-                                                         pack_bf16x2(yv[8 * q8 + 4], yv[8 * q8 + 5]),
-                                                         pack_bf16x2(yv[8 * q8 + 6], yv[8 * q8 + 7]));
-                            } else {
-                                float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.y) + off);
+                            for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(yv[2 * j], yv[2 * j + 1]);
+                        } else {
 #pragma unroll
-                                for (int q4 = 0; q4 < 4; ++q4)
-                                    dst[q4] = make_float4(yv[4 * q4], yv[4 * q4 + 1], yv[4 * q4 + 2],
-                                                          yv[4 * q4 + 3]);
-                                if constexpr (EPI == EPI_REQ) {
+                            for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(yv[j]);
+                            if constexpr (EPI == EPI_REQ) {
+                                // columns past N carry zero factors, so they add 0
+                                if (row_ok) {
 #pragma unroll
-                                    for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(yv[j]));
+                                    for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(yv[j]));
                                 }
                             }
                         }
+                    }
+                    if (lane == 0) bulk_wait_read_all();  // previous box of this warp has been read
+                    __syncwarp();
+                    stage_row_swizzled<RB>(stg, lane, w);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmY, stg_s, n0, mt * BM + quarter * 32);
+                        bulk_commit();
                     }
                 } else {
                     // thread owns output feature gm, columns = tokens n0 .. n0+CW-1
@@ -349,6 +383,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 if (row_ok) atomicMax(p.amax + gm, __float_as_uint(amax));
             }
         }
+        if (!SWAP && lane == 0) bulk_wait_all();  // this warp's TMA stores have landed
     }
 
     tc_fence_before();
@@ -359,41 +394,14 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 
 // ------------------------------------------------------------ host side
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
-                                             &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
-}
-
-// int8 matrix [rows, K] row-major; box = 128 bytes of K x box_rows rows,
-// 128-byte swizzle (matches sdesc_k_sw128); out-of-range elements read as 0.
-int make_tmap_i8(CUtensorMap* tm, const void* ptr, int64_t rows, int64_t K, int box_rows) {
-    auto fn = encode_fn();
-    if (!fn) return ZQ_ERR_CUDA;
-    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)K};
-    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box,
-                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? ZQ_OK : ZQ_ERR_CUDA;
-}
-
 constexpr int kMaxDevices = 64;
 
 template <int BN, int STAGES, bool SWAP, int EPI, int EW>
-int launch_cfg(const CUtensorMap& ta, const CUtensorMap& tb, const Params& p, const DeviceInfo& di,
-               cudaStream_t st) {
-    static_assert(smem_bytes<BN, STAGES>() <= 232448, "shared memory budget");
-    static_assert(smem_bytes<BN, STAGES>() > 116 * 1024, "one CTA per SM (TMEM ownership)");
+int launch_cfg(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ty, const Params& p,
+               const DeviceInfo& di, cudaStream_t st) {
+    constexpr size_t kSmem = smem_bytes<BN, STAGES, SWAP, EPI, EW>();
+    static_assert(kSmem <= 232448, "shared memory budget");
+    static_assert(kSmem > 116 * 1024, "one CTA per SM (TMEM ownership)");
     auto kern = w8a8_gemm_kernel<BN, STAGES, SWAP, EPI, EW>;
     static bool attr_set[kMaxDevices] = {};
     int dev = 0;
@@ -401,28 +409,37 @@ int launch_cfg(const CUtensorMap& ta, const CUtensorMap& tb, const Params& p, co
     if (dev < 0 || dev >= kMaxDevices) return ZQ_ERR_DEVICE;
     if (!attr_set[dev]) {
         int rc = cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                  (int)smem_bytes<BN, STAGES>()));
+                                                  (int)kSmem));
         if (rc) return rc;
         attr_set[dev] = true;
     }
     const int tiles = ((p.M + BM - 1) / BM) * ((p.N + BN - 1) / BN);
     const int grid = tiles < di.sm_count ? tiles : di.sm_count;
     count_launch();
-    kern<<<grid, block_threads<EW>(), smem_bytes<BN, STAGES>(), st>>>(ta, tb, p);
+    kern<<<grid, block_threads<EW>(), kSmem, st>>>(ta, tb, ty, p);
     return cuda_status(cudaGetLastError());
 }
 
-template <int BN, int STAGES, bool SWAP>
-int launch_epi(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const Params& p,
-               const DeviceInfo& di, cudaStream_t st) {
+// Pipeline depth: as many stages as fit beside the output staging boxes.
+template <int BN, bool SWAP, int EPI>
+constexpr int stages_for() {
+    if (SWAP) return 8;
+    if (BN == 256) return (EPI == EPI_BF16 || EPI == EPI_I32) ? 4 : 3;
+    if (BN == 192) return 4;
+    return 5;
+}
+
+template <int BN, bool SWAP>
+int launch_epi(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ty,
+               const Params& p, const DeviceInfo& di, cudaStream_t st) {
     // the epilogue is the long pole for short K loops: 16 warps (4 per SM
     // sub-partition) when it dequantizes, 8 for raw int32 and the decode shapes
     constexpr int EW = SWAP ? 8 : 16;
     switch (epi) {
-        case EPI_I32: return launch_cfg<BN, STAGES, SWAP, EPI_I32, 8>(ta, tb, p, di, st);
-        case EPI_F32: return launch_cfg<BN, STAGES, SWAP, EPI_F32, EW>(ta, tb, p, di, st);
-        case EPI_BF16: return launch_cfg<BN, STAGES, SWAP, EPI_BF16, EW>(ta, tb, p, di, st);
-        default: return launch_cfg<BN, STAGES, SWAP, EPI_REQ, EW>(ta, tb, p, di, st);
+        case EPI_I32: return launch_cfg<BN, stages_for<BN, SWAP, EPI_I32>(), SWAP, EPI_I32, 8>(ta, tb, ty, p, di, st);
+        case EPI_F32: return launch_cfg<BN, stages_for<BN, SWAP, EPI_F32>(), SWAP, EPI_F32, EW>(ta, tb, ty, p, di, st);
+        case EPI_BF16: return launch_cfg<BN, stages_for<BN, SWAP, EPI_BF16>(), SWAP, EPI_BF16, EW>(ta, tb, ty, p, di, st);
+        default: return launch_cfg<BN, stages_for<BN, SWAP, EPI_REQ>(), SWAP, EPI_REQ, EW>(ta, tb, ty, p, di, st);
     }
 }
 
@@ -447,6 +464,51 @@ int pick_bn(int64_t T, int64_t N, int sms) {
 }
 
 }  // namespace
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+int make_tmap_i8(CUtensorMap* tm, const void* ptr, int64_t rows, int64_t K, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return ZQ_ERR_CUDA;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K};
+    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box,
+                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ZQ_OK : ZQ_ERR_CUDA;
+}
+
+
+int make_tmap_out(CUtensorMap* tm, void* ptr, int64_t rows, int64_t cols, int esize) {
+    auto fn = encode_fn();
+    if (!fn) return ZQ_ERR_CUDA;
+    const CUtensorMapDataType dt = esize == 1   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                   : esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16
+                                                : CU_TENSOR_MAP_DATA_TYPE_UINT32;
+    const CUtensorMapSwizzle sw = esize == 1   ? CU_TENSOR_MAP_SWIZZLE_32B
+                                  : esize == 2 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                               : CU_TENSOR_MAP_SWIZZLE_128B;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(cols * esize)};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(tm, dt, 2, ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ZQ_OK : ZQ_ERR_CUDA;
+}
 
 int launch_w8a8_gemm(const LinearArgs& a, const DeviceInfo& di, cudaStream_t st) {
     int epi;
@@ -478,18 +540,22 @@ int launch_w8a8_gemm(const LinearArgs& a, const DeviceInfo& di, cudaStream_t st)
         const int bn = a.T <= 16 ? 16 : a.T <= 32 ? 32 : 64;
         if ((rc = make_tmap_i8(&ta, a.Wq, a.N, a.K, BM))) return rc;
         if ((rc = make_tmap_i8(&tb, a.xq, a.T, a.K, bn))) return rc;
-        if (bn == 16) return launch_epi<16, 8, true>(epi, ta, tb, p, di, st);
-        if (bn == 32) return launch_epi<32, 8, true>(epi, ta, tb, p, di, st);
-        return launch_epi<64, 8, true>(epi, ta, tb, p, di, st);
+        // the transposed output is written directly (ty is not used)
+        if (bn == 16) return launch_epi<16, true>(epi, ta, tb, ta, p, di, st);
+        if (bn == 32) return launch_epi<32, true>(epi, ta, tb, ta, p, di, st);
+        return launch_epi<64, true>(epi, ta, tb, ta, p, di, st);
     }
     p.M = (int)a.T;
     p.N = (int)a.N;
     const int bn = pick_bn(a.T, a.N, di.sm_count);
     if ((rc = make_tmap_i8(&ta, a.xq, a.T, a.K, BM))) return rc;
     if ((rc = make_tmap_i8(&tb, a.Wq, a.N, a.K, bn))) return rc;
-    if (bn == 256) return launch_epi<256, 4, false>(epi, ta, tb, p, di, st);
-    if (bn == 192) return launch_epi<192, 5, false>(epi, ta, tb, p, di, st);
-    return launch_epi<128, 6, false>(epi, ta, tb, p, di, st);
+    CUtensorMap ty;
+    if ((rc = make_tmap_out(&ty, p.y, a.T, a.N, epi == EPI_BF16 ? 2 : 4))) return rc;
+    // stages: as many as fit beside the output staging boxes
+    if (bn == 256) return launch_epi<256, false>(epi, ta, tb, ty, p, di, st);
+    if (bn == 192) return launch_epi<192, false>(epi, ta, tb, ty, p, di, st);
+    return launch_epi<128, false>(epi, ta, tb, ty, p, di, st);
 }
 
 }  // namespace zq

@@ -4,6 +4,7 @@
 // MMA, commit, TMEM loads).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -34,9 +35,27 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// exact-erf GeLU in fp32
-__device__ __forceinline__ float gelu_f(float v) {
-    return 0.5f * v * (1.0f + erff(v * 0.70710678118654752440f));
+// GeLU(x) = x * Phi(x), Phi the standard normal CDF, Phi(x) = (1 + erf(x/sqrt2))/2.
+// Branch-free: with u = |x|/sqrt2, the complementary error function is taken
+// from the rational approximation of Abramowitz & Stegun, Handbook of
+// Mathematical Functions, formula 7.1.26 (after Hastings):
+//   erfc(u) = (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-u^2),
+//   t = 1 / (1 + p u),  |error| <= 1.5e-7 for u >= 0;
+// Phi(-|x|) = erfc(u)/2 and Phi(|x|) = 1 - Phi(-|x|).  The coefficients below
+// are the published ones halved (folding the 1/2).
+__device__ __forceinline__ float gelu_f(float x) {
+    constexpr float kP = 0.3275911f;
+    constexpr float kA1 = 0.5f * 0.254829592f, kA2 = 0.5f * -0.284496736f, kA3 = 0.5f * 1.421413741f,
+                    kA4 = 0.5f * -1.453152027f, kA5 = 0.5f * 1.061405429f;
+    const float u = fabsf(x) * 0.70710678118654752f;
+    float t, e;
+    // hardware reciprocal and base-2 exponential (relative error about 2^-22):
+    // far below the 1.5e-7 of the approximation itself
+    asm("rcp.approx.f32 %0, %1;" : "=f"(t) : "f"(fmaf(kP, u, 1.0f)));
+    asm("ex2.approx.f32 %0, %1;" : "=f"(e) : "f"(x * x * -0.72134752044448170f));  // exp(-x^2/2)
+    const float poly = t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, kA5, kA4), kA3), kA2), kA1);
+    const float lower = poly * e;                             // Phi(-|x|)
+    return x * (x >= 0.0f ? 1.0f - lower : lower);
 }
 
 // Symmetric code: clamp(rint(y * inv), -127, 127).  The product is a single
@@ -213,6 +232,36 @@ __device__ __forceinline__ uint32_t quant4_packed_fused(uint64_t y01, uint64_t y
                        __byte_perm((uint32_t)m23, (uint32_t)(m23 >> 32), 0x0040), 0x5410);
 }
 
+// 2-D tiled bulk tensor store shared -> global (one thread), tracked as a
+// bulk async-group of the issuing thread.  Coordinates are never negative;
+// elements outside the tensor are not written.
+__device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src, int c0, int c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(src), "r"(c0), "r"(c1)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// until this thread's bulk stores have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// until this thread's bulk stores have completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Row `r` (0..31) of a 32-row staging box whose rows are RB bytes (32, 64 or
+// 128), written as RB/16 16-byte chunks at the positions the TMA swizzle of
+// the same width expects (32B, 64B, 128B modes): chunk j lands at
+// j ^ ((r >> s) & (RB/16 - 1)) with s = 2, 1, 0.  Eight consecutive rows then
+// cover all 32 banks, so the warp's writes are conflict-free.
+template <int RB>
+__device__ __forceinline__ void stage_row_swizzled(uint8_t* box, int r, const uint32_t* words) {
+    constexpr int NCH = RB / 16;
+    constexpr int SH = RB == 128 ? 0 : RB == 64 ? 1 : 2;
+    uint4* row = reinterpret_cast<uint4*>(box + r * RB);
+#pragma unroll
+    for (int j = 0; j < NCH; ++j)
+        row[j ^ ((r >> SH) & (NCH - 1))] = make_uint4(words[4 * j], words[4 * j + 1], words[4 * j + 2], words[4 * j + 3]);
+}
+
 // ---------------------------------------------------------------- tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
@@ -303,6 +352,81 @@ __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- clusters
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_count_x() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+    return r;
+}
+// shared::cta address -> the same offset in the shared memory of cluster CTA `rank`
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// bounded wait with cluster-scope acquire (data written by peer CTAs)
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                                  int* status, int site) {
+    if (mbar_try_wait_acq_cluster(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_try_wait_acq_cluster(bar, parity)) return true;
+        if ((n & 63u) == 0) {
+            if (abort_flag && *abort_flag) return false;
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                atomicCAS(status, 0, site);
+                if (abort_flag) *abort_flag = 1;
+                return false;
+            }
+        }
+    }
+}
+__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
+// every thread of every CTA of the cluster
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
@@ -366,9 +490,20 @@ struct LinearArgs {
     const float* bias;
     int act, out_kind;
     void* y;
-    float* h_ws;        // REQUANT: fp32 [T, N]
-    uint32_t* amax_ws;  // REQUANT: [T] absmax bit patterns
+    float* s_tok_out;   // REQUANT: new per-token scales [T]
+    float* h_ws;        // REQUANT (scratch path): fp32 [T, N]
+    uint32_t* amax_ws;  // REQUANT (scratch path): [T] absmax bit patterns
 };
 int launch_w8a8_gemm(const LinearArgs& a, const DeviceInfo& di, cudaStream_t st);
+// Requantizing linear with the per-token absmax exchanged between the CTAs of
+// a thread-block cluster (no scratch).  ZQ_ERR_SHAPE: shape not covered (the
+// caller then uses the scratch path).
+int launch_w8a8_requant_cluster(const LinearArgs& a, const DeviceInfo& di, cudaStream_t st);
+// int8 matrix [rows, K] as a TMA tensor: box 128 bytes of K x box_rows rows,
+// 128-byte swizzle, out-of-range elements read as 0.
+int make_tmap_i8(CUtensorMap* tm, const void* ptr, int64_t rows, int64_t K, int box_rows);
+// Output matrix [rows, cols] of `esize`-byte elements as a TMA store target:
+// box 32 columns x 32 rows, swizzle matching the 32*esize-byte box rows.
+int make_tmap_out(CUtensorMap* tm, void* ptr, int64_t rows, int64_t cols, int esize);
 
 }  // namespace zq
