@@ -346,11 +346,41 @@ def time_e2e(W, steps, warmup, torch):
 
 
 def count_launches(W, zq, torch):
-    before = zq.zq_launch_count()
-    for _, fn in W.stages:
+    """Kernels of this library launched per step, in total and per stage."""
+    per_stage = {}
+    for label, fn in W.stages:
+        before = zq.zq_launch_count()
         fn()
+        per_stage[label] = zq.zq_launch_count() - before
     torch.cuda.synchronize()
-    return zq.zq_launch_count() - before
+    return sum(per_stage.values()), per_stage
+
+
+def kernel_source_hash():
+    """Hash of the CUDA sources: ncu counters recorded for another version of
+    the kernels are not reported."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "w8a8_post_quantized_b200", "csrc", "*.cu*"))):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload, stage):
+    """DRAM bytes per launch of the stage's kernel from a committed ncu capture
+    (profiles/dram_traffic.json), if it was taken on the current sources."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(f"{workload}:{stage}")
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes")
 
 
 # ---------------------------------------------------------- CPU baseline
@@ -427,7 +457,7 @@ def main(argv=None):
     zq.lib()
 
     W = build_workload(a.workload, zq, torch, device)
-    launches_per_step = count_launches(W, zq, torch)
+    launches_per_step, stage_launches = count_launches(W, zq, torch)
     zq.zq_device_status()
 
     props = torch.cuda.get_device_properties(device)
@@ -447,24 +477,24 @@ def main(argv=None):
     peaks = load_peaks()
     int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
     stage_ms = {k: statistics.mean(v) for k, v in per_stage.items()}
-    # dominant kernel: the stage that is a single launch of the tcgen05 GEMM
-    # with the largest time (a quantizer when the workload has no GEMM)
-    gemm_stages = [k for k in stage_ms if k.startswith("linear")]
-    single = [k for k in gemm_stages if W.config.get("epilogue") != "gelu+requant" or k != "linear1"]
-    dom = max(single or gemm_stages or list(stage_ms), key=lambda k: stage_ms[k])
+    # dominant kernel: the longest stage that is a single launch of one kernel
+    single = [k for k in stage_ms if stage_launches.get(k) == 1]
+    dom = max(single or list(stage_ms), key=lambda k: stage_ms[k])
     bound, units, kind = W.kernel_units[dom]
     if bound == "tensor":
         achieved = units / (stage_ms[dom] * 1e-3) / 1e12
-        roof = {"kernel": f"w8a8_gemm ({dom})", "bound": "tensor", "achieved": round(achieved, 1),
+        roof = {"kernel": f"w8a8 linear ({dom})", "bound": "tensor", "achieved": round(achieved, 1),
                 "peak": round(int8_peak, 1), "unit": "TOPS", "frac": round(achieved / int8_peak, 4),
                 "peak_source": f"{peaks['source']} bf16 burst x {INT8_OVER_BF16:g} (nominal int8/bf16)",
-                "frac_vs_spec": round(achieved / SPEC_INT8_TOPS, 4), "traffic": None}
+                "frac_vs_spec": round(achieved / SPEC_INT8_TOPS, 4),
+                "traffic": recorded_traffic(a.workload, dom), "stage_ms": round(stage_ms[dom], 5)}
     else:
         achieved = units / (stage_ms[dom] * 1e-3) / 1e9
         roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "peak_source": f"{peaks['source']} copy bandwidth",
-                "frac_vs_spec": round(achieved / SPEC_HBM_GBS, 4), "traffic": None}
+                "frac_vs_spec": round(achieved / SPEC_HBM_GBS, 4),
+                "traffic": recorded_traffic(a.workload, dom), "stage_ms": round(stage_ms[dom], 5)}
     qlabel = "ln_quant" if "ln_quant" in stage_ms else "act_quant"
     qb = W.kernel_units[qlabel][1]
     q_gbs = qb / (stage_ms[qlabel] * 1e-3) / 1e9
@@ -494,6 +524,7 @@ def main(argv=None):
         "e2e": {"value": round(e2e_value, 3), "unit": unit, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": launches_per_step * a.steps,
+        "launches_per_stage": stage_launches,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not a.no_cpu_baseline and W.ops:
