@@ -68,8 +68,22 @@ struct Params {
     void* y;
     uint32_t* amax;     // EPI_REQ: per-token absmax bits
     int act;
+    int group_m;        // tile raster: groups of group_m row tiles sweep all column tiles
     int* status;
 };
+
+// Tile index -> (row tile, column tile).  Tiles run in groups of GM row tiles:
+// inside a group the row tile varies fastest, then the column tile, so the
+// group's slice of the M-side operand stays in L2 while every column tile
+// of the other operand streams past it once per group.
+__device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int GM, int& mt, int& nt) {
+    const int per_group = GM * n_tiles;
+    const int g = tile / per_group;
+    const int rem = tile - g * per_group;
+    const int gm = min(GM, m_tiles - g * GM);  // the last group may be short
+    mt = g * GM + rem % gm;
+    nt = rem / gm;
+}
 
 template <int BN>
 __host__ __device__ constexpr uint32_t tmem_cols() {
@@ -165,7 +179,8 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             uint32_t it = 0;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-                const int mt = tile % m_tiles, nt = tile / m_tiles;
+                int mt, nt;
+                tile_coords(tile, m_tiles, n_tiles, p.group_m, mt, nt);
                 for (int kb = 0; kb < kblocks; ++kb, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1u;
@@ -243,7 +258,8 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         float* st_b = stage_f + BN;             // per-column bias (non-swapped)
         uint32_t lt = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++lt) {
-            const int mt = tile % m_tiles, nt = tile / m_tiles;
+            int mt, nt;
+            tile_coords(tile, m_tiles, n_tiles, p.group_m, mt, nt);
             const int b = lt & 1;
             const uint32_t tph = (lt >> 1) & 1u;
             // stage the per-column factors of this tile (previous readers done)
@@ -444,17 +460,20 @@ int launch_epi(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const CUte
 }
 
 // Tile width for the non-swapped kernel: every CTA runs whole tiles, so the
-// time goes as (waves of tiles) x (tile width); take the cheapest, wider on
-// ties (fewer A re-reads, less shared-memory traffic per MMA).
+// time goes as (waves of tiles) x (tile width) / (efficiency of that width);
+// narrower tiles re-read A more often and feed the MMA less per byte
+// (measured on B200: 192 wide ~0.85, 128 wide ~0.7 of a 256-wide tile).
 int pick_bn(int64_t T, int64_t N, int sms) {
     const int cands[3] = {256, 192, 128};
+    const int64_t inv_eff_x20[3] = {20, 24, 29};  // 20 / efficiency
     int best = 256;
     int64_t best_cost = -1;
     const int64_t m_tiles = (T + BM - 1) / BM;
-    for (int bn : cands) {
+    for (int i = 0; i < 3; ++i) {
+        const int bn = cands[i];
         const int64_t tiles = m_tiles * ((N + bn - 1) / bn);
         const int64_t waves = (tiles + sms - 1) / sms;
-        const int64_t cost = waves * bn;
+        const int64_t cost = waves * bn * inv_eff_x20[i];
         if (best_cost < 0 || cost < best_cost) {
             best_cost = cost;
             best = bn;
@@ -529,6 +548,7 @@ int launch_w8a8_gemm(const LinearArgs& a, const DeviceInfo& di, cudaStream_t st)
     p.amax = a.amax_ws;
     p.act = a.act;
     p.status = di.status_word;
+    p.group_m = (int)((a.N + BM - 1) / BM);  // swapped: plain row-tile-fastest order
 
     const bool swap = a.T <= 64;
     CUtensorMap ta, tb;
@@ -548,6 +568,17 @@ int launch_w8a8_gemm(const LinearArgs& a, const DeviceInfo& di, cudaStream_t st)
     p.M = (int)a.T;
     p.N = (int)a.N;
     const int bn = pick_bn(a.T, a.N, di.sm_count);
+    {
+        // row tiles per raster group: their activation slice (128 rows x K
+        // bytes each) within ~24 MB of L2, at least one wave's worth of rows
+        const int64_t m_tiles = (a.T + BM - 1) / BM;
+        int64_t gm = (24ll << 20) / ((int64_t)BM * a.K);
+        const int64_t n_tiles = (a.N + bn - 1) / bn;
+        const int64_t min_gm = (di.sm_count + n_tiles - 1) / n_tiles;
+        if (gm < min_gm) gm = min_gm;
+        if (gm < 1) gm = 1;
+        p.group_m = (int)(gm < m_tiles ? gm : m_tiles);
+    }
     if ((rc = make_tmap_i8(&ta, a.xq, a.T, a.K, BM))) return rc;
     if ((rc = make_tmap_i8(&tb, a.Wq, a.N, a.K, bn))) return rc;
     CUtensorMap ty;

@@ -431,14 +431,13 @@ int launch_typed(const Tin* x, int64_t T, int64_t H, const float* gamma, const f
     const Shape sh = kShapes[idx];
     const int teams = sh.block / sh.tpr;
     const int row_bytes = (int)(H * sizeof(Tin));
-    // rows per stage: about kStageTarget bytes, a multiple of the team count;
-    // fewer rows per stage when the problem is too small to give every SM
-    // a few stages of work (idle teams are fine then)
+    // rows per stage: about kStageTarget bytes and a multiple of the team
+    // count (every team busy); fewer rows per stage, down to one per team,
+    // when the problem is too small to give every SM a few stages of work
     int R = kStageTarget / row_bytes;
     R = R < teams ? teams : R - R % teams;
     const int64_t want_units = 2 * (int64_t)di.sm_count;
-    while (R > 1 && (T + R - 1) / R < want_units) R = R > teams ? R - teams : R / 2;
-    if (R < 1) R = 1;
+    while (R > teams && (T + R - 1) / R < want_units) R -= teams;
     const int stage_bytes = R * row_bytes;
     const int n_par = LN ? 2 : (bias ? 1 : 0);
     const size_t par_bytes = idx < kFirstGlobalParamShape ? (size_t)n_par * H * sizeof(float) : 0;
