@@ -100,8 +100,10 @@ __host__ __device__ constexpr size_t smem_bytes() {
     // epilogue warp, non-swapped only) + barriers/flags + per-column factors
     // (bf16 outputs stage only the per-column scale; their bias is read
     // through L1, which leaves room for a fourth pipeline stage at BN = 256)
-    return 1024 + (size_t)STAGES * (A_STAGE + BN * BK) + (SWAP ? 0 : (size_t)EW * 32 * out_row_bytes<EPI>()) +
-           256 + (EPI == EPI_I32 ? 0 : EPI == EPI_BF16 && !SWAP ? 1 : 2) * BN * sizeof(float);
+    // (swapped kernels: two int32 partial-accumulator buffers for split-K)
+    return 1024 + (size_t)STAGES * (A_STAGE + BN * BK) +
+           (SWAP ? (size_t)2 * BM * BN * 4 : (size_t)EW * 32 * out_row_bytes<EPI>()) + 256 +
+           (EPI == EPI_I32 ? 0 : EPI == EPI_BF16 && !SWAP ? 1 : 2) * BN * sizeof(float);
 }
 
 template <int BN, int STAGES, bool SWAP, int EPI, int EW>
@@ -125,7 +127,9 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const uint32_t sA = base;
     const uint32_t sB = base + STAGES * A_STAGE;
     const uint32_t sStg = sB + STAGES * B_STAGE;  // 1024-aligned: every stage is a multiple of 1024
-    const uint32_t sBar = sStg + STG_BYTES;
+    // swapped: split-K partials [2 buffers][BM rows][BN] int32 (in place of the staging boxes)
+    const uint32_t sPart = sStg;
+    const uint32_t sBar = sStg + (SWAP ? 2u * BM * BN * 4u : STG_BYTES);
     uint8_t* gBar = gbase + (sBar - base);
     // barrier layout: full[S], empty[S], tfull[2], tempty[2], drain
     auto bar_full = [&](int s) { return sBar + 8u * s; };
@@ -133,12 +137,21 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     auto bar_tfull = [&](int b) { return sBar + 8u * (2 * STAGES + b); };
     auto bar_tempty = [&](int b) { return sBar + 8u * (2 * STAGES + 2 + b); };
     const uint32_t bar_drain = sBar + 8u * (2 * STAGES + 4);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gBar + 8 * (2 * STAGES + 5));
+    // split-K (swapped): partials of buffer b are ready at the leader / free again at a peer
+    auto bar_red_full = [&](int b) { return sBar + 8u * (2 * STAGES + 5 + b); };
+    auto bar_red_free = [&](int b) { return sBar + 8u * (2 * STAGES + 7 + b); };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gBar + 8 * (2 * STAGES + 9));
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     float* stage_f = reinterpret_cast<float*>(gBar + 256);  // [2][BN]
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    // swapped kernels run as clusters of S CTAs splitting K (S may be 1);
+    // the others as independent CTAs
+    const int S = SWAP ? (int)cluster_size() : 1;
+    const int rank = SWAP ? (int)cluster_ctarank() : 0;
+    const int cl = SWAP ? (int)cluster_id_x() : (int)blockIdx.x;
+    const int ncl = SWAP ? (int)cluster_count_x() : (int)gridDim.x;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -148,6 +161,10 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar_tfull(b), 1);
             mbar_init(bar_tempty(b), EW);
+            if (SWAP) {
+                mbar_init(bar_red_full(b), S > 1 ? S - 1 : 1);
+                mbar_init(bar_red_free(b), 1);
+            }
         }
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
@@ -166,22 +183,26 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (SWAP) cluster_sync_all();  // peers' barriers initialised before any remote arrive
     const uint32_t tmem_base = *tmem_slot;
 
     const int m_tiles = (p.M + BM - 1) / BM;
     const int n_tiles = (p.N + BN - 1) / BN;
     const int num_tiles = m_tiles * n_tiles;
-    const int kblocks = (p.K + BK - 1) / BK;
+    const int kblocks_all = (p.K + BK - 1) / BK;
+    // this CTA's share of the K loop (the whole loop unless split)
+    const int kb_begin = rank * kblocks_all / S;
+    const int kb_end = (rank + 1) * kblocks_all / S;
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
             uint32_t it = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+            for (int tile = cl; ok && tile < num_tiles; tile += ncl) {
                 int mt, nt;
                 tile_coords(tile, m_tiles, n_tiles, p.group_m, mt, nt);
-                for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1u;
                     if (!mbar_wait(bar_empty(s), ph ^ 1u, abort_flag, p.status, SITE_PRODUCER_EMPTY)) {
@@ -206,7 +227,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         if (lane == 0) {
             uint32_t it = 0, lt = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++lt) {
+            for (int tile = cl; ok && tile < num_tiles; tile += ncl, ++lt) {
                 const int b = lt & 1;
                 const uint32_t tph = (lt >> 1) & 1u;
                 if (!mbar_wait(bar_tempty(b), tph ^ 1u, abort_flag, p.status, SITE_MMA_TMEM_EMPTY)) {
@@ -215,7 +236,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(b * BN);
-                for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1u;
                     if (!mbar_wait(bar_full(s), ph, abort_flag, p.status, SITE_MMA_FULL)) {
@@ -229,7 +250,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     for (int k = 0; k < BK / UMMA_K; ++k)
                         // +32 bytes along K inside the swizzle atom = +2 in the
                         // descriptor's (address >> 4) field
-                        mma_i8(d_tmem, da + 2u * k, db + 2u * k, IDESC, (kb | k) != 0 ? 1u : 0u);
+                        mma_i8(d_tmem, da + 2u * k, db + 2u * k, IDESC, (kb > kb_begin || k > 0) ? 1u : 0u);
                     mma_commit(bar_empty(s));  // stage free once these MMAs finish
                 }
                 if (ok) mma_commit(bar_tfull(b));  // accumulator b complete
@@ -257,11 +278,42 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         float* st_a = stage_f;                  // per-column scale (or token scale when swapped)
         float* st_b = stage_f + BN;             // per-column bias (non-swapped)
         uint32_t lt = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++lt) {
+        for (int tile = cl; tile < num_tiles; tile += ncl, ++lt) {
             int mt, nt;
             tile_coords(tile, m_tiles, n_tiles, p.group_m, mt, nt);
             const int b = lt & 1;
             const uint32_t tph = (lt >> 1) & 1u;
+            if constexpr (SWAP) {
+                if (S > 1 && rank > 0) {
+                    // split-K helper: export this slice's partial accumulators to
+                    // shared memory for the leader, once the leader has consumed
+                    // the previous use of buffer b
+                    const bool fr = mbar_wait(bar_red_free(b), tph ^ 1u, abort_flag, p.status, SITE_EPI_TMEM_FULL);
+                    const bool tf = fr && mbar_wait(bar_tfull(b), tph, abort_flag, p.status, SITE_EPI_TMEM_FULL);
+                    if (!named_bar_and(1, kEpiThreads, tf)) break;
+                    tc_fence_after();
+                    const uint32_t t_row = tmem_base + (uint32_t)(b * BN) + ((uint32_t)(quarter * 32) << 16);
+                    int32_t* part = reinterpret_cast<int32_t*>(gbase + (sPart - base)) + (b * BM + r) * BN;
+#pragma unroll 1
+                    for (int c = c_begin; c < c_end; ++c) {
+                        uint32_t v[CW];
+                        if constexpr (CW == 32) tmem_ld_32x32b_x32(t_row + c * CW, v);
+                        else tmem_ld_32x32b_x16(t_row + c * CW, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int q4 = 0; q4 < CW / 4; ++q4)
+                            reinterpret_cast<int4*>(part + c * CW)[q4] =
+                                make_int4((int)v[4 * q4], (int)v[4 * q4 + 1], (int)v[4 * q4 + 2], (int)v[4 * q4 + 3]);
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar_tempty(b));
+                    fence_acq_rel_cluster();
+                    named_bar_sync(1, kEpiThreads);
+                    if (et == 0) mbar_arrive_cluster(mapa_shared(bar_red_full(b), 0u));
+                    continue;
+                }
+            }
             // stage the per-column factors of this tile (previous readers done)
             named_bar_sync(1, kEpiThreads);
             for (int i = et; EPI != EPI_I32 && i < BN; i += kEpiThreads) {
@@ -278,7 +330,9 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             named_bar_sync(1, kEpiThreads);
             // all 128 epilogue threads take the same decision (barrier with an
             // AND-reduction), so none is left behind at a later barrier
-            const bool got = mbar_wait(bar_tfull(b), tph, abort_flag, p.status, SITE_EPI_TMEM_FULL);
+            bool got = mbar_wait(bar_tfull(b), tph, abort_flag, p.status, SITE_EPI_TMEM_FULL);
+            if (SWAP && S > 1)  // split-K leader: the other slices' partials are in
+                got = got && mbar_wait_cluster(bar_red_full(b), tph, abort_flag, p.status, SITE_EPI_TMEM_FULL);
             if (!named_bar_and(1, kEpiThreads, got)) break;
             tc_fence_after();
 
@@ -303,6 +357,21 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 if constexpr (CW == 32) tmem_ld_32x32b_x32(t_row + c * CW, v);
                 else tmem_ld_32x32b_x16(t_row + c * CW, v);
                 tmem_ld_wait();
+                if (SWAP && S > 1) {
+                    // exact int32 sum of the K slices: peers' partials over DSMEM
+                    const uint32_t own = sPart + (uint32_t)((b * BM + r) * BN + c * CW) * 4u;
+                    for (int q = 1; q < S; ++q) {
+                        const uint32_t src = mapa_shared(own, (uint32_t)q);
+#pragma unroll
+                        for (int q4 = 0; q4 < CW / 4; ++q4) {
+                            const int4 t4 = ld_cluster_v4(src + 16u * q4);
+                            v[4 * q4] += (uint32_t)t4.x;
+                            v[4 * q4 + 1] += (uint32_t)t4.y;
+                            v[4 * q4 + 2] += (uint32_t)t4.z;
+                            v[4 * q4 + 3] += (uint32_t)t4.w;
+                        }
+                    }
+                }
                 const int n0 = nt * BN + c * CW;   // first N-side index of the chunk
                 if constexpr (!SWAP) {
                     // thread owns token gm (box row `lane`), columns n0 .. n0+31; the
@@ -395,6 +464,12 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_tempty(b));
+            if (SWAP && S > 1) {
+                // the peers' partial buffers b have been read: hand them back
+                named_bar_sync(1, kEpiThreads);
+                if (et == 0)
+                    for (int q = 1; q < S; ++q) mbar_arrive_cluster(mapa_shared(bar_red_free(b), (uint32_t)q));
+            }
             if constexpr (EPI == EPI_REQ && !SWAP) {
                 if (row_ok) atomicMax(p.amax + gm, __float_as_uint(amax));
             }
@@ -404,6 +479,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 
     tc_fence_before();
     __syncthreads();
+    if (SWAP) cluster_sync_all();  // no CTA leaves while a peer may still read its shared memory
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
 }
@@ -411,6 +487,33 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 // ------------------------------------------------------------ host side
 
 constexpr int kMaxDevices = 64;
+
+// Largest number of co-resident clusters of `S` CTAs for this kernel (cached).
+template <typename K>
+int max_clusters(K kern, int S, size_t smem, int threads, int dev) {
+    static int cache[kMaxDevices][9] = {};
+    if (S < 1 || S > 8) return 0;
+    if (cache[dev][S] == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = S;
+        at[0].val.clusterDim.y = 1;
+        at[0].val.clusterDim.z = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        cfg.gridDim = dim3(S);
+        cfg.blockDim = dim3(threads);
+        cfg.dynamicSmemBytes = smem;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            n = -1;
+        }
+        cache[dev][S] = n;
+    }
+    return cache[dev][S];
+}
 
 template <int BN, int STAGES, bool SWAP, int EPI, int EW>
 int launch_cfg(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ty, const Params& p,
@@ -430,16 +533,51 @@ int launch_cfg(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& 
         attr_set[dev] = true;
     }
     const int tiles = ((p.M + BM - 1) / BM) * ((p.N + BN - 1) / BN);
-    const int grid = tiles < di.sm_count ? tiles : di.sm_count;
-    count_launch();
-    kern<<<grid, block_threads<EW>(), kSmem, st>>>(ta, tb, ty, p);
-    return cuda_status(cudaGetLastError());
+    if constexpr (SWAP) {
+        // split K over a cluster of S CTAs: S minimising (rounds of tiles) / S,
+        // with a small charge per extra slice; each slice keeps >= 1 k-block
+        const int kblocks = (p.K + BK - 1) / BK;
+        int bestS = 1, bestN = 0;
+        double best = 1e30;
+        for (int S = 1; S <= 8 && S <= kblocks; ++S) {
+            const int n = max_clusters(kern, S, kSmem, block_threads<EW>(), dev);
+            if (n < 1) continue;
+            const int ncl = n < tiles ? n : tiles;
+            const int rounds = (tiles + ncl - 1) / ncl;
+            const double cost = (double)rounds / S + 0.03 * (S - 1);
+            if (cost < best) {
+                best = cost;
+                bestS = S;
+                bestN = ncl;
+            }
+        }
+        if (bestN < 1) return ZQ_ERR_CUDA;
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = bestS;
+        at[0].val.clusterDim.y = 1;
+        at[0].val.clusterDim.z = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        cfg.gridDim = dim3(bestN * bestS);
+        cfg.blockDim = dim3(block_threads<EW>());
+        cfg.dynamicSmemBytes = kSmem;
+        cfg.stream = st;
+        count_launch();
+        return cuda_status(cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, p));
+    } else {
+        const int grid = tiles < di.sm_count ? tiles : di.sm_count;
+        count_launch();
+        kern<<<grid, block_threads<EW>(), kSmem, st>>>(ta, tb, ty, p);
+        return cuda_status(cudaGetLastError());
+    }
 }
 
 // Pipeline depth: as many stages as fit beside the output staging boxes.
 template <int BN, bool SWAP, int EPI>
 constexpr int stages_for() {
-    if (SWAP) return 8;
+    if (SWAP) return BN == 64 ? 6 : 8;  // beside the split-K partial buffers
     if (BN == 256) return (EPI == EPI_BF16 || EPI == EPI_I32) ? 4 : 3;
     if (BN == 192) return 4;
     return 5;
