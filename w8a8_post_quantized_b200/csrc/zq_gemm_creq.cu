@@ -14,11 +14,13 @@
 // block of 128 rows and all N columns: CTA `rank` computes column tiles
 // 2*rank and 2*rank+1 into its two TMEM accumulators (512 columns, the whole
 // TMEM).  The epilogue
-//   pass 1  dequantizes, adds bias, applies GeLU, writes the fp32 result back
-//           into TMEM in place (tcgen05.st) and keeps a per-row partial absmax;
+//   pass 1  dequantizes, adds bias, applies GeLU (packed fp32 pair arithmetic),
+//           writes the fp32 result back into TMEM in place (tcgen05.st) and
+//           keeps a per-row partial absmax;
 //   xchg    pushes each row's partial absmax into every cluster CTA's shared
-//           memory (distributed shared memory stores) and arrives on each
-//           CTA's exchange mbarrier; waits for all C partials of its own rows;
+//           memory with asynchronous distributed-shared-memory stores that
+//           count their bytes on the receiver's exchange mbarrier; waits until
+//           all C partials of its own rows have landed;
 //   pass 2  reads the fp32 result back from TMEM and writes int8 codes with
 //           scale = absmax/127, code = rint(fl(h * fl(127/absmax))).
 // The producer (TMA) and MMA warps are those of the plain kernel; the tile
@@ -62,16 +64,53 @@ struct Params {
     int* status;
 };
 
-template <int STAGES>
+template <int STAGES, int NSTG>
 __host__ __device__ constexpr size_t smem_bytes() {
-    // ring + int8 output staging (one 32x32 box per epilogue warp) + barriers/
+    // ring + int8 output staging (NSTG 32x32 boxes per epilogue warp) + barriers/
     // flags (256) + column factors [2 halves][scale, bias][BN] + per-slice row
     // partials [4][BM] + exchange [2][kMaxCluster][BM]
-    return 1024 + (size_t)STAGES * (A_STAGE + B_STAGE) + EW * 32 * 32 + 256 + 2 * 2 * BN * 4 + 4 * BM * 4 +
+    return 1024 + (size_t)STAGES * (A_STAGE + B_STAGE) + NSTG * EW * 32 * 32 + 256 + 2 * 2 * BN * 4 + 4 * BM * 4 +
            2 * kMaxCluster * BM * 4;
 }
 
-template <int STAGES>
+// Pass 1 on one 32-column chunk of one row, in place: accumulators (int32
+// words) in, y = s_tok * s_grp * acc + bias (+GeLU) as fp32 words out, in
+// packed pair arithmetic.  UNI: the chunk lies in one weight group, so the
+// combined scale is one number.
+template <bool GELU, bool UNI>
+__device__ __forceinline__ void pass1_chunk(uint32_t (&v)[32], float row_scale, const float* scc,
+                                            const float* bic, float& pmax) {
+    uint32_t bad = 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        v[j] += 0x4B400000u;  // 1.5*2^23 + acc as a float, when |acc| < 2^22
+        bad |= v[j] ^ 0x4B000000u;
+    }
+    uint64_t f[16];
+    if (bad & kI2fBadMask) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            f[i] = f2_pack((float)(int)(v[2 * i] - 0x4B400000u), (float)(int)(v[2 * i + 1] - 0x4B400000u));
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) f[i] = f2_sub(u2_pack(v[2 * i], v[2 * i + 1]), f2_splat(12582912.0f));
+    }
+    const uint64_t rs2 = f2_splat(row_scale);
+    const uint64_t a_uni = f2_splat(row_scale * scc[0]);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const uint64_t a2 = UNI ? a_uni : f2_mul(rs2, *reinterpret_cast<const uint64_t*>(scc + 2 * i));
+        uint64_t t = f2_fma(a2, f[i], *reinterpret_cast<const uint64_t*>(bic + 2 * i));
+        if (GELU) t = gelu2(t);
+        float t0, t1;
+        f2_unpack(t, t0, t1);
+        pmax = fmaxf(pmax, fmaxf(fabsf(t0), fabsf(t1)));
+        v[2 * i] = __float_as_uint(t0);
+        v[2 * i + 1] = __float_as_uint(t1);
+    }
+}
+
+template <int STAGES, int NSTG>
 __global__ void __launch_bounds__(kThreads, 1)
 w8a8_requant_cluster_kernel(const __grid_constant__ CUtensorMap tmA,
                             const __grid_constant__ CUtensorMap tmB,
@@ -83,8 +122,8 @@ w8a8_requant_cluster_kernel(const __grid_constant__ CUtensorMap tmA,
     uint8_t* gbase = smem_raw + (base - raw);
     const uint32_t sA = base;
     const uint32_t sB = base + STAGES * A_STAGE;
-    const uint32_t sStg = sB + STAGES * B_STAGE;  // [EW][32 rows][32 B], 1024-aligned
-    const uint32_t sBar = sStg + EW * 32 * 32;
+    const uint32_t sStg = sB + STAGES * B_STAGE;  // [EW][NSTG][32 rows][32 B], 1024-aligned
+    const uint32_t sBar = sStg + NSTG * EW * 32 * 32;
     uint8_t* gBar = gbase + (sBar - base);
     // barriers: full[S], empty[S], tfull[2], tempty[2], drain, xbar[2]
     auto bar_full = [&](int s) { return sBar + 8u * s; };
@@ -118,7 +157,7 @@ w8a8_requant_cluster_kernel(const __grid_constant__ CUtensorMap tmA,
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar_tfull(b), 1);
             mbar_init(bar_tempty(b), EW);
-            mbar_init(bar_xchg(b), p.C);   // one arrival per cluster CTA
+            mbar_init(bar_xchg(b), 1);     // the local expect-tx arrival; peers' bytes complete it
         }
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
@@ -214,8 +253,9 @@ w8a8_requant_cluster_kernel(const __grid_constant__ CUtensorMap tmA,
         const int c_begin = slice * CT / SLICES, c_end = (slice + 1) * CT / SLICES;
         const int r = quarter * 32 + lane;
         const int et = threadIdx.x - 64;
-        uint8_t* stg = gbase + (sStg - base) + (uint32_t)(warp - 2) * 32u * 32u;  // this warp's box
-        const uint32_t stg_s = smem_u32(stg);
+        uint8_t* stg0 = gbase + (sStg - base) + (uint32_t)(warp - 2) * NSTG * 32u * 32u;  // this warp's boxes
+        const bool gelu = p.act == ZQ_ACT_GELU;
+        const bool uni = p.G % CW == 0;  // every 32-column chunk lies in one weight group
         uint32_t mbi = 0;
         bool alive = true;
         for (int mb = cl; alive && mb < m_tiles; mb += ncl, ++mbi) {
@@ -251,12 +291,14 @@ w8a8_requant_cluster_kernel(const __grid_constant__ CUtensorMap tmA,
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(t_row + c * CW, v);
                     tmem_ld_wait();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        float t = fmaf(row_scale * sc[c * CW + j], (float)(int)v[j], bi[c * CW + j]);
-                        if (p.act == ZQ_ACT_GELU) t = gelu_f(t);
-                        pmax = fmaxf(pmax, fabsf(t));
-                        v[j] = __float_as_uint(t);
+                    const float* scc = sc + c * CW;
+                    const float* bic = bi + c * CW;
+                    if (gelu) {
+                        if (uni) pass1_chunk<true, true>(v, row_scale, scc, bic, pmax);
+                        else pass1_chunk<true, false>(v, row_scale, scc, bic, pmax);
+                    } else {
+                        if (uni) pass1_chunk<false, true>(v, row_scale, scc, bic, pmax);
+                        else pass1_chunk<false, false>(v, row_scale, scc, bic, pmax);
                     }
                     tmem_st_32x32b_x32(t_row + c * CW, v);
                 }
@@ -265,20 +307,25 @@ w8a8_requant_cluster_kernel(const __grid_constant__ CUtensorMap tmA,
             if (!alive) break;
 
             // exchange: row absmax over this CTA's column slices, then over the cluster
+            // Each CTA's exchange barrier expects C * BM * 4 bytes per use; every
+            // cluster CTA sends its BM row partials with asynchronous stores that
+            // count on the receiver's barrier.  Buffer `buf` is rewritten two row
+            // blocks later, by which time every receiver has read it: a sender
+            // gets there only after its own barrier for the next block completed,
+            // which needs every CTA's next-block partials, sent after reading.
             const int buf = mbi & 1;
             slice_part[slice * BM + r] = pmax;
+            if (et == 0) mbar_arrive_expect_tx(bar_xchg(buf), (uint32_t)(p.C * BM * 4));
             named_bar_sync(1, kEpiThreads);
             if (slice == 0) {
                 float m = slice_part[r];
 #pragma unroll
                 for (int s = 1; s < SLICES; ++s) m = fmaxf(m, slice_part[s * BM + r]);
                 const uint32_t local = smem_u32(xch + (buf * kMaxCluster + rank) * BM + r);
-                for (int q = 0; q < p.C; ++q) st_cluster_u32(mapa_shared(local, (uint32_t)q), __float_as_uint(m));
-                fence_acq_rel_cluster();
+                for (int q = 0; q < p.C; ++q)
+                    st_async_u32(mapa_shared(local, (uint32_t)q), __float_as_uint(m),
+                                 mapa_shared(bar_xchg(buf), (uint32_t)q));
             }
-            named_bar_sync(1, kEpiThreads);
-            if (et == 0)
-                for (int q = 0; q < p.C; ++q) mbar_arrive_cluster(mapa_shared(bar_xchg(buf), (uint32_t)q));
             const bool got = mbar_wait_cluster(bar_xchg(buf), (mbi >> 1) & 1u, abort_flag, p.status, SITE_E_XCHG);
             if (!named_bar_and(1, kEpiThreads, got)) break;
             float amax = 0.0f;
@@ -288,7 +335,8 @@ w8a8_requant_cluster_kernel(const __grid_constant__ CUtensorMap tmA,
             if (rank == 0 && slice == 0 && row_ok) p.s_tok_out[gm] = scale;
 
             // pass 2: codes from the fp32 values kept in TMEM
-            const float magic = 12582912.0f;  // 1.5 * 2^23: fl(t + magic) holds rint(t)
+            const uint64_t inv2 = f2_splat(inv);  // codes: fl(fl(h * inv) + 1.5*2^23), two roundings
+            int kst = 0;                       // staging box in turn
             for (int h = 0; h < 2; ++h) {
                 if (!(h ? real1 : real0)) continue;
                 const uint32_t t_row = tmem_base + (uint32_t)(h * BN) + ((uint32_t)(quarter * 32) << 16);
@@ -300,17 +348,18 @@ w8a8_requant_cluster_kernel(const __grid_constant__ CUtensorMap tmA,
                     const int n0 = (2 * rank + h) * BN + c * CW;
                     uint32_t w[8];
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        uint32_t b4[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            b4[e] = __float_as_uint(__fadd_rn(__fmul_rn(__uint_as_float(v[4 * q + e]), inv), magic));
-                        w[q] = __byte_perm(__byte_perm(b4[0], b4[1], 0x0040), __byte_perm(b4[2], b4[3], 0x0040),
-                                           0x5410);
-                    }
+                    for (int q = 0; q < 8; ++q)
+                        w[q] = quant4_packed(u2_pack(v[4 * q], v[4 * q + 1]), u2_pack(v[4 * q + 2], v[4 * q + 3]), inv2);
                     // the warp's 32x32 box of codes: shared memory, then one TMA store
-                    // (rows >= M and columns >= N are clipped)
-                    if (lane == 0) bulk_wait_read_all();
+                    // (rows >= M and columns >= N are clipped); the box's previous
+                    // store (NSTG boxes ago) must have finished reading it
+                    uint8_t* stg = stg0 + kst * 32 * 32;
+                    const uint32_t stg_s = smem_u32(stg);
+                    kst = kst + 1 == NSTG ? 0 : kst + 1;
+                    if (lane == 0) {
+                        if (NSTG == 2) bulk_wait_read_1();
+                        else bulk_wait_read_all();
+                    }
                     __syncwarp();
                     stage_row_swizzled<32>(stg, lane, w);
                     fence_proxy_async_smem();
@@ -336,21 +385,22 @@ w8a8_requant_cluster_kernel(const __grid_constant__ CUtensorMap tmA,
 }
 
 constexpr int kStages = 4;
+constexpr int kStg = 1;
 constexpr int kMaxDevices = 64;
 
 }  // namespace
 
 int launch_w8a8_requant_cluster(const LinearArgs& a, const DeviceInfo& di, cudaStream_t st) {
-    static_assert(smem_bytes<kStages>() <= 232448, "shared memory budget");
-    static_assert(smem_bytes<kStages>() > 116 * 1024, "one CTA per SM (TMEM ownership)");
+    static_assert(smem_bytes<kStages, kStg>() <= 232448, "shared memory budget");
+    static_assert(smem_bytes<kStages, kStg>() > 116 * 1024, "one CTA per SM (TMEM ownership)");
     const int64_t n_tiles = (a.N + BN - 1) / BN;
     const int C = (int)((n_tiles + 1) / 2);
     if (a.T <= 64 || C < 1 || C > kMaxCluster) return ZQ_ERR_SHAPE;
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= kMaxDevices) return ZQ_ERR_DEVICE;
-    auto kern = w8a8_requant_cluster_kernel<kStages>;
-    const size_t smem = smem_bytes<kStages>();
+    auto kern = w8a8_requant_cluster_kernel<kStages, kStg>;
+    const size_t smem = smem_bytes<kStages, kStg>();
     static bool attr_set[kMaxDevices] = {};
     static int max_clusters[kMaxDevices][kMaxCluster + 1] = {};
     int rc;

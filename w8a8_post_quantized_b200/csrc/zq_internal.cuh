@@ -50,9 +50,11 @@ __device__ __forceinline__ float gelu_f(float x) {
     const float u = fabsf(x) * 0.70710678118654752f;
     float t, e;
     // hardware reciprocal and base-2 exponential (relative error about 2^-22):
-    // far below the 1.5e-7 of the approximation itself
-    asm("rcp.approx.f32 %0, %1;" : "=f"(t) : "f"(fmaf(kP, u, 1.0f)));
-    asm("ex2.approx.f32 %0, %1;" : "=f"(e) : "f"(x * x * -0.72134752044448170f));  // exp(-x^2/2)
+    // far below the 1.5e-7 of the approximation itself.  Flushing subnormals
+    // is harmless: the reciprocal's argument is >= 1 and an exponential below
+    // 2^-126 leaves Phi(-|x|) far under one ulp of the result.
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t) : "f"(fmaf(kP, u, 1.0f)));
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(x * x * -0.72134752044448170f));  // exp(-x^2/2)
     const float poly = t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, kA5, kA4), kA3), kA2), kA1);
     const float lower = poly * e;                             // Phi(-|x|)
     return x * (x >= 0.0f ? 1.0f - lower : lower);
@@ -199,6 +201,55 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
     return r;
 }
 
+__device__ __forceinline__ uint64_t f2_splat(float v) { return f2_pack(v, v); }
+// two 32-bit words as one 64-bit register pair, lo first
+__device__ __forceinline__ uint64_t u2_pack(uint32_t lo, uint32_t hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+    return r;
+}
+
+// GeLU of a pair of values in packed fp32 arithmetic, the approximation of
+// gelu_f rearranged to need no select: with a = |x| and L = Phi(-a),
+//   gelu(x) = x * Phi(x) = max(x, 0) - a * L
+// (x >= 0: x - x L;  x < 0: x * Phi(x) = x * Phi(-a) = -a L).  L is the
+// Abramowitz & Stegun 7.1.26 form t P(t) exp(-a^2/2) / 2, t = 1/(1 + p a/sqrt2);
+// the coefficients enter negated and halved so that the last step is one
+// fused multiply-add: gelu = max(x, 0) + (t Q(t) a) exp(-a^2/2), Q = -P/2.
+__device__ __forceinline__ uint64_t gelu2(uint64_t x2) {
+    constexpr float kPs = 0.3275911f * 0.70710678118654752f;
+    constexpr float kB1 = -0.5f * 0.254829592f, kB2 = -0.5f * -0.284496736f, kB3 = -0.5f * 1.421413741f,
+                    kB4 = -0.5f * -1.453152027f, kB5 = -0.5f * 1.061405429f;
+    float x0, x1;
+    f2_unpack(x2, x0, x1);
+    const uint64_t a2 = f2_pack(fabsf(x0), fabsf(x1));
+    float d0, d1, q0, q1, t0, t1, e0, e1;
+    f2_unpack(f2_fma(a2, f2_splat(kPs), f2_splat(1.0f)), d0, d1);
+    f2_unpack(f2_mul(f2_mul(a2, f2_splat(-0.72134752044448170f)), a2), q0, q1);  // -a^2/2 * log2(e)
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t0) : "f"(d0));
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t1) : "f"(d1));
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e0) : "f"(q0));
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e1) : "f"(q1));
+    const uint64_t t2 = f2_pack(t0, t1);
+    uint64_t h = f2_fma(t2, f2_splat(kB5), f2_splat(kB4));
+    h = f2_fma(t2, h, f2_splat(kB3));
+    h = f2_fma(t2, h, f2_splat(kB2));
+    h = f2_fma(t2, h, f2_splat(kB1));
+    const uint64_t ta = f2_mul(t2, a2);
+    return f2_fma(f2_mul(h, ta), f2_pack(e0, e1), f2_pack(fmaxf(x0, 0.0f), fmaxf(x1, 0.0f)));
+}
+
+// Exact int32 -> fp32 of a pair without the conversion unit, for |v| < 2^22:
+// the word 0x4B400000 + v is the float 1.5*2^23 + v, and subtracting 1.5*2^23
+// is exact.  `bad` accumulates a word whose bits 23..31 are all zero exactly
+// when every converted v was in range (0x4B400000 + v within [2^23, 2^24)).
+__device__ __forceinline__ uint64_t i2f2_magic(uint32_t v0, uint32_t v1, uint32_t& bad) {
+    const uint32_t w0 = v0 + 0x4B400000u, w1 = v1 + 0x4B400000u;
+    bad |= (w0 ^ 0x4B000000u) | (w1 ^ 0x4B000000u);
+    return f2_sub(u2_pack(w0, w1), f2_splat(12582912.0f));
+}
+constexpr uint32_t kI2fBadMask = 0xFF800000u;
+
 // Codes of four fp32 values packed little-endian into one word.
 // t = fl(y * inv) as a packed multiply; then fl(t + 1.5*2^23) (a scalar add
 // with explicit round-to-nearest, which is never contracted with the multiply)
@@ -244,6 +295,8 @@ __device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src, int
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // until this thread's bulk stores have finished reading shared memory
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// until at most one of this thread's bulk store groups is still reading shared memory
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 // until this thread's bulk stores have completed
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
@@ -389,6 +442,13 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
 }
 __device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
     asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+// Asynchronous 4-byte store into a cluster peer's shared memory that counts
+// its bytes on the peer's mbarrier (complete-tx); both addresses from mapa.
+__device__ __forceinline__ void st_async_u32(uint32_t cluster_addr, uint32_t v, uint32_t cluster_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.u32 [%0], %1, [%2];" ::"r"(cluster_addr),
+                 "r"(v), "r"(cluster_bar)
+                 : "memory");
 }
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
