@@ -14,14 +14,17 @@ Metric: INT8 tera-operations per second of the whole step (2*T*N*K integer
 ops per GEMM, summed, over the step time), with the fused LN/token-quant
 bandwidth and the per-kernel roofline alongside.
 
-Timing: each stage is one CUDA graph of the library's C-ABI calls; every
+Timing: each step is one CUDA graph of the library's C-ABI calls (the
+kernels chained by programmatic dependent launch); every
 timed step is preceded by an L2 flush -- a 256 MiB write followed by a read
 of the same buffer, so the 126 MB L2 ends up holding only clean lines of the
 flush buffer and no write-back of flush data lands inside the timed step --
 and is bracketed by CUDA events on the launching stream (the flush is
 outside the events).  W >= 3 warm-up steps; K timed steps; barrier + synchronize on both
 sides; the maximum over ranks.  Multi-GPU runs are independent replicas
-(the path needs no exchange): value = ops of all ranks / max time.
+(the path needs no exchange): value = ops of all ranks / max time.  The
+per-stage breakdown and the roofline come from a second timed run with one
+graph per stage (each stage then pays its own launch latency).
 
 --impl reference times the CPU oracle (the plain C reference of the same
 path) on the host cores, on a bounded sample of the same workload.
@@ -266,8 +269,14 @@ def build_workload(name, zq, torch, device):
 # ------------------------------------------------------------------ timing
 
 def time_device(W, steps, warmup, torch):
-    """Per-stage CUDA graphs; flush L2 before each step; CUDA events around
-    each stage on the launching stream.  Returns per-step and per-stage ms."""
+    """Flush L2 before each step; CUDA events on the launching stream.
+
+    The step time comes from one CUDA graph holding the whole step (its
+    kernels chained by programmatic dependent launch, as a serving loop would
+    replay them).  The per-stage times come from a second timed run in which
+    every stage is its own graph with events between them; they include each
+    stage's own launch latency, so they are upper bounds on the kernels.
+    Returns per-step ms and per-stage ms lists."""
     stream = torch.cuda.current_stream()
     flush = L2Flush(torch, W.device)
     for _, fn in W.stages:       # eager warm-up (sets kernel attributes, loads modules)
@@ -282,11 +291,24 @@ def time_device(W, steps, warmup, torch):
             with torch.cuda.graph(g, stream=cap):
                 fn()
             graphs.append((label, g))
+        whole = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(whole, stream=cap):
+            for _, fn in W.stages:
+                fn()
     stream.wait_stream(cap)
     torch.cuda.synchronize()
     n = len(graphs)
 
-    def run(k, record):
+    def run_step(k):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(k)]
+        for s in range(k):
+            flush()
+            evs[s][0].record(stream)
+            whole.replay()
+            evs[s][1].record(stream)
+        return evs
+
+    def run_stages(k):
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(k)]
         for s in range(k):
             flush()
@@ -296,16 +318,20 @@ def time_device(W, steps, warmup, torch):
                 evs[s][i + 1].record(stream)
         return evs
 
-    run(warmup, False)
+    run_step(warmup)
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
-    evs = run(steps, True)
+    evs = run_step(steps)
     torch.cuda.synchronize()
     barrier()
-    per_step = [e[0].elapsed_time(e[-1]) for e in evs]
+    per_step = [a.elapsed_time(b) for a, b in evs]
+    run_stages(warmup)
+    torch.cuda.synchronize()
+    evs = run_stages(steps)
+    torch.cuda.synchronize()
     per_stage = {label: [e[i].elapsed_time(e[i + 1]) for e in evs] for i, (label, _) in enumerate(graphs)}
-    del graphs
+    del graphs, whole
     return per_step, per_stage
 
 
@@ -515,7 +541,7 @@ def main(argv=None):
         "data": "synthetic (seeded; layer shapes only, random weights)",
         "config": dict(W.config, parallelism=f"replicas x{world}",
                        l2="flushed before every timed step (256 MiB write + read-back)",
-                       timing="per-stage CUDA graphs, CUDA events on the launching stream"),
+                       timing="one CUDA graph per step (kernels chained by programmatic dependent launch), CUDA events on the launching stream; per-stage times from per-stage graphs"),
         "tokens_per_s": round(world * W.tokens / (ms_per_step * 1e-3), 1),
         "stages_ms": {k: round(v, 5) for k, v in stage_ms.items()},
         "ln_quant_gbs": round(q_gbs, 1),

@@ -2,6 +2,7 @@
 // of it on the host, before anything is enqueued), per-device facts, the
 // device status word used by bounded waits, and the entry points.
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <atomic>
@@ -20,6 +21,14 @@ static thread_local char t_last_error[256] = "no error";
 static std::atomic<uint64_t> g_launches{0};
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+int pdl_attr(cudaLaunchAttribute& attr) {
+    static const bool off = getenv("ZQ_NO_PDL") != nullptr;
+    if (off) return 0;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    return 1;
+}
 
 void set_cuda_error(cudaError_t e) {
     snprintf(t_last_error, sizeof(t_last_error), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));

@@ -184,6 +184,8 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     if (SWAP) cluster_sync_all();  // peers' barriers initialised before any remote arrive
+    griddep_wait();                // inputs and outputs are free of the previous grid in the stream
+    griddep_launch_dependents();
     const uint32_t tmem_base = *tmem_slot;
 
     const int m_tiles = (p.M + BM - 1) / BM;
@@ -553,13 +555,13 @@ int launch_cfg(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& 
         }
         if (bestN < 1) return ZQ_ERR_CUDA;
         cudaLaunchConfig_t cfg = {};
-        cudaLaunchAttribute at[1];
+        cudaLaunchAttribute at[2];
         at[0].id = cudaLaunchAttributeClusterDimension;
         at[0].val.clusterDim.x = bestS;
         at[0].val.clusterDim.y = 1;
         at[0].val.clusterDim.z = 1;
         cfg.attrs = at;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = 1 + (unsigned)pdl_attr(at[1]);
         cfg.gridDim = dim3(bestN * bestS);
         cfg.blockDim = dim3(block_threads<EW>());
         cfg.dynamicSmemBytes = kSmem;
@@ -568,9 +570,16 @@ int launch_cfg(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& 
         return cuda_status(cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, p));
     } else {
         const int grid = tiles < di.sm_count ? tiles : di.sm_count;
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute at[1];
+        cfg.attrs = at;
+        cfg.numAttrs = (unsigned)pdl_attr(at[0]);
+        cfg.gridDim = dim3((unsigned)grid);
+        cfg.blockDim = dim3(block_threads<EW>());
+        cfg.dynamicSmemBytes = kSmem;
+        cfg.stream = st;
         count_launch();
-        kern<<<grid, block_threads<EW>(), kSmem, st>>>(ta, tb, ty, p);
-        return cuda_status(cudaGetLastError());
+        return cuda_status(cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, p));
     }
 }
 

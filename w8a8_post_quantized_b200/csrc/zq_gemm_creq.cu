@@ -177,6 +177,8 @@ w8a8_requant_cluster_kernel(const __grid_constant__ CUtensorMap tmA,
     __syncthreads();
     tc_fence_after();
     cluster_sync_all();  // every CTA's exchange barriers are initialised before any peer arrives
+    griddep_wait();      // inputs and outputs are free of the previous grid in the stream
+    griddep_launch_dependents();
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 0) {
@@ -410,7 +412,7 @@ int launch_w8a8_requant_cluster(const LinearArgs& a, const DeviceInfo& di, cudaS
         attr_set[dev] = true;
     }
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = C;
     attr[0].val.clusterDim.y = 1;
@@ -434,6 +436,7 @@ int launch_w8a8_requant_cluster(const LinearArgs& a, const DeviceInfo& di, cudaS
     const int64_t m_tiles = (a.T + BM - 1) / BM;
     const int ncl = (int)(m_tiles < max_clusters[dev][C] ? m_tiles : max_clusters[dev][C]);
     cfg.gridDim = dim3(ncl * C);
+    cfg.numAttrs = 1 + (unsigned)pdl_attr(attr[1]);
 
     CUtensorMap ta, tb, ty;
     if ((rc = make_tmap_i8(&ta, a.xq, a.T, a.K, BM))) return rc;

@@ -443,6 +443,17 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
 __device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
     asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
+// Programmatic dependent launch.  griddep_wait: block until every grid this
+// one depends on has completed and its memory is visible (immediate when the
+// launch has no such dependency).  griddep_launch_dependents: this CTA no
+// longer holds back the launch of the next grid in the stream; that grid's
+// CTAs then take free SMs and wait in griddep_wait, so its launch latency and
+// prologue overlap this grid's tail.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Asynchronous 4-byte store into a cluster peer's shared memory that counts
 // its bytes on the peer's mbarrier (complete-tx); both addresses from mapa.
 __device__ __forceinline__ void st_async_u32(uint32_t cluster_addr, uint32_t v, uint32_t cluster_bar) {
@@ -535,6 +546,11 @@ int device_info(DeviceInfo* out);  // returns zq_status
 
 void set_cuda_error(cudaError_t e);
 void count_launch();  // every kernel launch goes through this
+// Programmatic dependent launch for the hot-path kernels: fills `attr` with
+// the stream-serialization attribute (returns 1) unless ZQ_NO_PDL is set in
+// the environment (returns 0).  Kernels launched with it call griddep_wait()
+// before touching global memory.
+int pdl_attr(cudaLaunchAttribute& attr);
 int cuda_status(cudaError_t e);  // ZQ_OK or ZQ_ERR_CUDA (and records the text)
 
 // launchers (no validation; the C ABI validates)

@@ -215,6 +215,8 @@ rowq_pipe_kernel(const Tin* __restrict__ x, int T, int H, float inv_h, int R, in
         fence_proxy_async_smem();
         fence_barrier_init();
     }
+    griddep_wait();  // inputs and outputs are free of the previous grid in the stream
+    griddep_launch_dependents();
     if constexpr (SMEMP) {
         const float* src0 = LN ? gamma : bias;
         constexpr int QPP = NP / 2;  // 16-byte quarters per piece
@@ -450,10 +452,17 @@ int launch_typed(const Tin* x, int64_t T, int64_t H, const float* gamma, const f
     auto kern = pipe_kernel<Tin, LN>(idx);
     int rc = cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     if (rc) return rc;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    cfg.attrs = at;
+    cfg.numAttrs = (unsigned)pdl_attr(at[0]);
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)sh.block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
     count_launch();
-    kern<<<grid, sh.block, smem, st>>>(x, (int)T, (int)H, 1.0f / (float)H, R, nstages, gamma, beta,
-                                       eps, bias, act, q, s_tok, di.status_word);
-    return cuda_status(cudaGetLastError());
+    return cuda_status(cudaLaunchKernelEx(&cfg, kern, x, (int)T, (int)H, 1.0f / (float)H, R, nstages, gamma, beta,
+                                          eps, bias, act, q, s_tok, di.status_word));
 }
 
 }  // namespace
