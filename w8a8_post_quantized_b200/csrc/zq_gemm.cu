@@ -277,105 +277,62 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const uint32_t stg_s = smem_u32(stg);
         (void)stg;
         (void)stg_s;
-        float* st_a = stage_f;                  // per-column scale (or token scale when swapped)
-        float* st_b = stage_f + BN;             // per-column bias (non-swapped)
-        uint32_t lt = 0;
-        for (int tile = cl; tile < num_tiles; tile += ncl, ++lt) {
-            int mt, nt;
-            tile_coords(tile, m_tiles, n_tiles, p.group_m, mt, nt);
-            const int b = lt & 1;
-            const uint32_t tph = (lt >> 1) & 1u;
-            if constexpr (SWAP) {
-                if (S > 1 && rank > 0) {
-                    // split-K helper: export this slice's partial accumulators to
-                    // shared memory for the leader, once the leader has consumed
-                    // the previous use of buffer b
-                    const bool fr = mbar_wait(bar_red_free(b), tph ^ 1u, abort_flag, p.status, SITE_EPI_TMEM_FULL);
-                    const bool tf = fr && mbar_wait(bar_tfull(b), tph, abort_flag, p.status, SITE_EPI_TMEM_FULL);
-                    if (!named_bar_and(1, kEpiThreads, tf)) break;
-                    tc_fence_after();
-                    const uint32_t t_row = tmem_base + (uint32_t)(b * BN) + ((uint32_t)(quarter * 32) << 16);
-                    int32_t* part = reinterpret_cast<int32_t*>(gbase + (sPart - base)) + (b * BM + r) * BN;
-#pragma unroll 1
-                    for (int c = c_begin; c < c_end; ++c) {
-                        uint32_t v[CW];
-                        if constexpr (CW == 32) tmem_ld_32x32b_x32(t_row + c * CW, v);
-                        else tmem_ld_32x32b_x16(t_row + c * CW, v);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int q4 = 0; q4 < CW / 4; ++q4)
-                            reinterpret_cast<int4*>(part + c * CW)[q4] =
-                                make_int4((int)v[4 * q4], (int)v[4 * q4 + 1], (int)v[4 * q4 + 2], (int)v[4 * q4 + 3]);
-                    }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar_tempty(b));
-                    fence_acq_rel_cluster();
-                    named_bar_sync(1, kEpiThreads);
-                    if (et == 0) mbar_arrive_cluster(mapa_shared(bar_red_full(b), 0u));
-                    continue;
-                }
-            }
-            // stage the per-column factors of this tile (previous readers done)
-            named_bar_sync(1, kEpiThreads);
-            for (int i = et; EPI != EPI_I32 && i < BN; i += kEpiThreads) {
-                const int n = nt * BN + i;
+        const bool gelu = p.act == ZQ_ACT_GELU;
+        if constexpr (!SWAP) {
+            // Each warp runs on its own (no CTA-wide barrier per tile): it waits
+            // for the accumulator, converts its chunks and frees the accumulator
+            // with its own arrival.  The column factors of the next chunk it will
+            // handle (lane l: scale and bias of column l) and the token scale of
+            // its next tile are loaded one step ahead, so their latency hides
+            // behind the current chunk.
+            const bool uni = p.G % 32 == 0;  // each 32-column chunk lies in one weight group
+            float pa = 0.0f, pb = 0.0f, prs = 0.0f;
+            auto fetch_cols = [&](int tile, int c) {
+                int mt_, nt_;
+                tile_coords(tile, m_tiles, n_tiles, p.group_m, mt_, nt_);
+                const int n = nt_ * BN + c * CW + lane;
                 const bool in = n < p.N;
-                if constexpr (SWAP) {
-                    st_a[i] = (EPI != EPI_I32 && in) ? __ldg(p.s_tok + n) : 0.0f;
-                } else {
-                    st_a[i] = (EPI != EPI_I32 && in) ? __ldg(p.s_grp + n / p.G) : 0.0f;
-                    if constexpr (EPI != EPI_BF16)
-                        st_b[i] = (EPI != EPI_I32 && in && p.bias) ? __ldg(p.bias + n) : 0.0f;
-                }
+                pa = in ? __ldg(p.s_grp + n / p.G) : 0.0f;
+                pb = (in && p.bias) ? __ldg(p.bias + n) : 0.0f;
+            };
+            auto fetch_row = [&](int tile) {
+                int mt_, nt_;
+                tile_coords(tile, m_tiles, n_tiles, p.group_m, mt_, nt_);
+                const int gm = mt_ * BM + r;
+                prs = gm < p.M ? __ldg(p.s_tok + gm) : 0.0f;
+            };
+            if (EPI != EPI_I32 && cl < num_tiles) {
+                fetch_cols(cl, c_begin);
+                fetch_row(cl);
             }
-            named_bar_sync(1, kEpiThreads);
-            // all 128 epilogue threads take the same decision (barrier with an
-            // AND-reduction), so none is left behind at a later barrier
-            bool got = mbar_wait(bar_tfull(b), tph, abort_flag, p.status, SITE_EPI_TMEM_FULL);
-            if (SWAP && S > 1)  // split-K leader: the other slices' partials are in
-                got = got && mbar_wait_cluster(bar_red_full(b), tph, abort_flag, p.status, SITE_EPI_TMEM_FULL);
-            if (!named_bar_and(1, kEpiThreads, got)) break;
-            tc_fence_after();
-
-            const int gm = mt * BM + r;          // M-side row owned by this thread
-            const bool row_ok = gm < p.M;
-            float row_scale = 0.0f, row_bias = 0.0f;
-            if (EPI != EPI_I32 && row_ok) {
-                if constexpr (SWAP) {
-                    row_scale = __ldg(p.s_grp + gm / p.G);
-                    row_bias = p.bias ? __ldg(p.bias + gm) : 0.0f;
-                } else {
-                    row_scale = __ldg(p.s_tok + gm);
-                }
-            }
-            float amax = 0.0f;
-            const uint32_t t_row = tmem_base + (uint32_t)(b * BN) + ((uint32_t)(quarter * 32) << 16);
-            static_assert(SWAP || CW == 32, "non-swapped tiles are whole 32-column chunks");
-
+            uint32_t lt = 0;
+            for (int tile = cl; tile < num_tiles; tile += ncl, ++lt) {
+                int mt, nt;
+                tile_coords(tile, m_tiles, n_tiles, p.group_m, mt, nt);
+                const int b = lt & 1;
+                const uint32_t tph = (lt >> 1) & 1u;
+                const float row_scale = prs;
+                if (EPI != EPI_I32 && tile + ncl < num_tiles) fetch_row(tile + ncl);
+                // the warp's lanes take one decision, so none waits alone later
+                const bool got = mbar_wait(bar_tfull(b), tph, abort_flag, p.status, SITE_EPI_TMEM_FULL);
+                if (!__all_sync(0xFFFFFFFFu, got)) break;
+                tc_fence_after();
+                const int gm = mt * BM + r;  // token row owned by this thread
+                const bool row_ok = gm < p.M;
+                float amax = 0.0f;
+                const uint32_t t_row = tmem_base + (uint32_t)(b * BN) + ((uint32_t)(quarter * 32) << 16);
+                static_assert(SWAP || CW == 32, "non-swapped tiles are whole 32-column chunks");
 #pragma unroll 1
-            for (int c = c_begin; c < c_end; ++c) {
-                uint32_t v[CW];
-                if constexpr (CW == 32) tmem_ld_32x32b_x32(t_row + c * CW, v);
-                else tmem_ld_32x32b_x16(t_row + c * CW, v);
-                tmem_ld_wait();
-                if (SWAP && S > 1) {
-                    // exact int32 sum of the K slices: peers' partials over DSMEM
-                    const uint32_t own = sPart + (uint32_t)((b * BM + r) * BN + c * CW) * 4u;
-                    for (int q = 1; q < S; ++q) {
-                        const uint32_t src = mapa_shared(own, (uint32_t)q);
-#pragma unroll
-                        for (int q4 = 0; q4 < CW / 4; ++q4) {
-                            const int4 t4 = ld_cluster_v4(src + 16u * q4);
-                            v[4 * q4] += (uint32_t)t4.x;
-                            v[4 * q4 + 1] += (uint32_t)t4.y;
-                            v[4 * q4 + 2] += (uint32_t)t4.z;
-                            v[4 * q4 + 3] += (uint32_t)t4.w;
-                        }
+                for (int c = c_begin; c < c_end; ++c) {
+                    const float ca = pa, cb = pb;
+                    if (EPI != EPI_I32) {
+                        if (c + 1 < c_end) fetch_cols(tile, c + 1);
+                        else if (tile + ncl < num_tiles) fetch_cols(tile + ncl, c_begin);
                     }
-                }
-                const int n0 = nt * BN + c * CW;   // first N-side index of the chunk
-                if constexpr (!SWAP) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(t_row + c * CW, v);
+                    tmem_ld_wait();
+                    const int n0 = nt * BN + c * CW;  // first column of the chunk
                     // thread owns token gm (box row `lane`), columns n0 .. n0+31; the
                     // warp's 32x32 box goes through shared memory to one TMA store
                     // (rows >= M and columns >= N are clipped by the store)
@@ -384,45 +341,30 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 #pragma unroll
                         for (int j = 0; j < 32; ++j) w[j] = v[j];
                     } else {
-                        float yv[32];
-                        // bf16 outputs read this chunk's bias through L1 (zero past N
-                        // or without bias); the others use the staged copy
-                        const bool has_b = EPI == EPI_BF16 && p.bias != nullptr && n0 < p.N;
-                        const float4* b4 = reinterpret_cast<const float4*>(p.bias + (has_b ? n0 : 0));
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            float be[4];
-                            if constexpr (EPI == EPI_BF16) {
-                                const float4 t4 = (has_b && n0 + 4 * q < p.N) ? __ldg(b4 + q)
-                                                                               : make_float4(0.f, 0.f, 0.f, 0.f);
-                                be[0] = t4.x;
-                                be[1] = t4.y;
-                                be[2] = t4.z;
-                                be[3] = t4.w;
-                            } else {
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) be[e] = st_b[c * CW + 4 * q + e];
-                            }
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int j = 4 * q + e;
-                                float t = fmaf(row_scale * st_a[c * CW + j], (float)(int)v[j], be[e]);
-                                if (p.act == ZQ_ACT_GELU) t = gelu_f(t);
-                                yv[j] = t;
-                            }
+                        uint64_t f[16];
+                        if (gelu) {
+                            if (uni) dequant_chunk_lanes<true, true>(v, row_scale, ca, cb, f);
+                            else dequant_chunk_lanes<true, false>(v, row_scale, ca, cb, f);
+                        } else {
+                            if (uni) dequant_chunk_lanes<false, true>(v, row_scale, ca, cb, f);
+                            else dequant_chunk_lanes<false, false>(v, row_scale, ca, cb, f);
                         }
                         if constexpr (EPI == EPI_BF16) {
 #pragma unroll
-                            for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(yv[2 * j], yv[2 * j + 1]);
+                            for (int i = 0; i < 16; ++i) {
+                                float t0, t1;
+                                f2_unpack(f[i], t0, t1);
+                                w[i] = pack_bf16x2(t0, t1);
+                            }
                         } else {
 #pragma unroll
-                            for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(yv[j]);
-                            if constexpr (EPI == EPI_REQ) {
+                            for (int i = 0; i < 16; ++i) {
+                                float t0, t1;
+                                f2_unpack(f[i], t0, t1);
+                                w[2 * i] = __float_as_uint(t0);
+                                w[2 * i + 1] = __float_as_uint(t1);
                                 // columns past N carry zero factors, so they add 0
-                                if (row_ok) {
-#pragma unroll
-                                    for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(yv[j]));
-                                }
+                                if (EPI == EPI_REQ && row_ok) amax = fmaxf(amax, fmaxf(fabsf(t0), fabsf(t1)));
                             }
                         }
                     }
@@ -435,7 +377,103 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         tma_store_2d(&tmY, stg_s, n0, mt * BM + quarter * 32);
                         bulk_commit();
                     }
-                } else {
+                }
+                // accumulator b may be overwritten once every epilogue warp has read it
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_tempty(b));
+                if constexpr (EPI == EPI_REQ) {
+                    if (row_ok) atomicMax(p.amax + gm, __float_as_uint(amax));
+                }
+            }
+            if (lane == 0) bulk_wait_all();  // this warp's TMA stores have landed
+        } else {
+            float* st_a = stage_f;                  // per-column scale (or token scale when swapped)
+            uint32_t lt = 0;
+            for (int tile = cl; tile < num_tiles; tile += ncl, ++lt) {
+                int mt, nt;
+                tile_coords(tile, m_tiles, n_tiles, p.group_m, mt, nt);
+                const int b = lt & 1;
+                const uint32_t tph = (lt >> 1) & 1u;
+                if constexpr (SWAP) {
+                    if (S > 1 && rank > 0) {
+                        // split-K helper: export this slice's partial accumulators to
+                        // shared memory for the leader, once the leader has consumed
+                        // the previous use of buffer b
+                        const bool fr = mbar_wait(bar_red_free(b), tph ^ 1u, abort_flag, p.status, SITE_EPI_TMEM_FULL);
+                        const bool tf = fr && mbar_wait(bar_tfull(b), tph, abort_flag, p.status, SITE_EPI_TMEM_FULL);
+                        if (!named_bar_and(1, kEpiThreads, tf)) break;
+                        tc_fence_after();
+                        const uint32_t t_row = tmem_base + (uint32_t)(b * BN) + ((uint32_t)(quarter * 32) << 16);
+                        int32_t* part = reinterpret_cast<int32_t*>(gbase + (sPart - base)) + (b * BM + r) * BN;
+    #pragma unroll 1
+                        for (int c = c_begin; c < c_end; ++c) {
+                            uint32_t v[CW];
+                            if constexpr (CW == 32) tmem_ld_32x32b_x32(t_row + c * CW, v);
+                            else tmem_ld_32x32b_x16(t_row + c * CW, v);
+                            tmem_ld_wait();
+    #pragma unroll
+                            for (int q4 = 0; q4 < CW / 4; ++q4)
+                                reinterpret_cast<int4*>(part + c * CW)[q4] =
+                                    make_int4((int)v[4 * q4], (int)v[4 * q4 + 1], (int)v[4 * q4 + 2], (int)v[4 * q4 + 3]);
+                        }
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar_tempty(b));
+                        fence_acq_rel_cluster();
+                        named_bar_sync(1, kEpiThreads);
+                        if (et == 0) mbar_arrive_cluster(mapa_shared(bar_red_full(b), 0u));
+                        continue;
+                    }
+                }
+                // stage the per-column factors of this tile (previous readers done)
+                named_bar_sync(1, kEpiThreads);
+                for (int i = et; EPI != EPI_I32 && i < BN; i += kEpiThreads) {
+                    const int n = nt * BN + i;
+                    const bool in = n < p.N;
+                    st_a[i] = (EPI != EPI_I32 && in) ? __ldg(p.s_tok + n) : 0.0f;
+                }
+                named_bar_sync(1, kEpiThreads);
+                // all 128 epilogue threads take the same decision (barrier with an
+                // AND-reduction), so none is left behind at a later barrier
+                bool got = mbar_wait(bar_tfull(b), tph, abort_flag, p.status, SITE_EPI_TMEM_FULL);
+                if (SWAP && S > 1)  // split-K leader: the other slices' partials are in
+                    got = got && mbar_wait_cluster(bar_red_full(b), tph, abort_flag, p.status, SITE_EPI_TMEM_FULL);
+                if (!named_bar_and(1, kEpiThreads, got)) break;
+                tc_fence_after();
+
+                const int gm = mt * BM + r;          // M-side row owned by this thread
+                const bool row_ok = gm < p.M;
+                float row_scale = 0.0f, row_bias = 0.0f;
+                if (EPI != EPI_I32 && row_ok) {
+                    row_scale = __ldg(p.s_grp + gm / p.G);
+                    row_bias = p.bias ? __ldg(p.bias + gm) : 0.0f;
+                }
+                const uint32_t t_row = tmem_base + (uint32_t)(b * BN) + ((uint32_t)(quarter * 32) << 16);
+                static_assert(SWAP || CW == 32, "non-swapped tiles are whole 32-column chunks");
+
+    #pragma unroll 1
+                for (int c = c_begin; c < c_end; ++c) {
+                    uint32_t v[CW];
+                    if constexpr (CW == 32) tmem_ld_32x32b_x32(t_row + c * CW, v);
+                    else tmem_ld_32x32b_x16(t_row + c * CW, v);
+                    tmem_ld_wait();
+                    if (SWAP && S > 1) {
+                        // exact int32 sum of the K slices: peers' partials over DSMEM
+                        const uint32_t own = sPart + (uint32_t)((b * BM + r) * BN + c * CW) * 4u;
+                        for (int q = 1; q < S; ++q) {
+                            const uint32_t src = mapa_shared(own, (uint32_t)q);
+    #pragma unroll
+                            for (int q4 = 0; q4 < CW / 4; ++q4) {
+                                const int4 t4 = ld_cluster_v4(src + 16u * q4);
+                                v[4 * q4] += (uint32_t)t4.x;
+                                v[4 * q4 + 1] += (uint32_t)t4.y;
+                                v[4 * q4 + 2] += (uint32_t)t4.z;
+                                v[4 * q4 + 3] += (uint32_t)t4.w;
+                            }
+                        }
+                    }
+                    const int n0 = nt * BN + c * CW;   // first N-side index of the chunk
                     // thread owns output feature gm, columns = tokens n0 .. n0+CW-1
 #pragma unroll
                     for (int j = 0; j < CW; ++j) {
@@ -461,22 +499,18 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         else static_cast<float*>(p.y)[off] = t;
                     }
                 }
-            }
-            // accumulator b may be overwritten once all four warps have read it
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_tempty(b));
-            if (SWAP && S > 1) {
-                // the peers' partial buffers b have been read: hand them back
-                named_bar_sync(1, kEpiThreads);
-                if (et == 0)
-                    for (int q = 1; q < S; ++q) mbar_arrive_cluster(mapa_shared(bar_red_free(b), (uint32_t)q));
-            }
-            if constexpr (EPI == EPI_REQ && !SWAP) {
-                if (row_ok) atomicMax(p.amax + gm, __float_as_uint(amax));
+                // accumulator b may be overwritten once all four warps have read it
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_tempty(b));
+                if (SWAP && S > 1) {
+                    // the peers' partial buffers b have been read: hand them back
+                    named_bar_sync(1, kEpiThreads);
+                    if (et == 0)
+                        for (int q = 1; q < S; ++q) mbar_arrive_cluster(mapa_shared(bar_red_free(b), (uint32_t)q));
+                }
             }
         }
-        if (!SWAP && lane == 0) bulk_wait_all();  // this warp's TMA stores have landed
     }
 
     tc_fence_before();

@@ -80,30 +80,12 @@ __host__ __device__ constexpr size_t smem_bytes() {
 template <bool GELU, bool UNI>
 __device__ __forceinline__ void pass1_chunk(uint32_t (&v)[32], float row_scale, const float* scc,
                                             const float* bic, float& pmax) {
-    uint32_t bad = 0;
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-        v[j] += 0x4B400000u;  // 1.5*2^23 + acc as a float, when |acc| < 2^22
-        bad |= v[j] ^ 0x4B000000u;
-    }
     uint64_t f[16];
-    if (bad & kI2fBadMask) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-            f[i] = f2_pack((float)(int)(v[2 * i] - 0x4B400000u), (float)(int)(v[2 * i + 1] - 0x4B400000u));
-    } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) f[i] = f2_sub(u2_pack(v[2 * i], v[2 * i + 1]), f2_splat(12582912.0f));
-    }
-    const uint64_t rs2 = f2_splat(row_scale);
-    const uint64_t a_uni = f2_splat(row_scale * scc[0]);
+    dequant_chunk<GELU, UNI>(v, row_scale, scc, bic, nullptr, 0, f);
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-        const uint64_t a2 = UNI ? a_uni : f2_mul(rs2, *reinterpret_cast<const uint64_t*>(scc + 2 * i));
-        uint64_t t = f2_fma(a2, f[i], *reinterpret_cast<const uint64_t*>(bic + 2 * i));
-        if (GELU) t = gelu2(t);
         float t0, t1;
-        f2_unpack(t, t0, t1);
+        f2_unpack(f[i], t0, t1);
         pmax = fmaxf(pmax, fmaxf(fabsf(t0), fabsf(t1)));
         v[2 * i] = __float_as_uint(t0);
         v[2 * i + 1] = __float_as_uint(t1);

@@ -250,6 +250,83 @@ __device__ __forceinline__ uint64_t i2f2_magic(uint32_t v0, uint32_t v1, uint32_
 }
 constexpr uint32_t kI2fBadMask = 0xFF800000u;
 
+// 32 int32 accumulators -> 16 packed fp32 pairs, exact: the conversion-unit
+// free path when every |acc| < 2^22, else the hardware conversion.  `v` is
+// modified (offset words) on return.
+__device__ __forceinline__ void acc32_to_f2(uint32_t (&v)[32], uint64_t (&f)[16]) {
+    uint32_t bad = 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        v[j] += 0x4B400000u;  // 1.5*2^23 + acc as a float, when |acc| < 2^22
+        bad |= v[j] ^ 0x4B000000u;
+    }
+    if (bad & kI2fBadMask) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            f[i] = f2_pack((float)(int)(v[2 * i] - 0x4B400000u), (float)(int)(v[2 * i + 1] - 0x4B400000u));
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) f[i] = f2_sub(u2_pack(v[2 * i], v[2 * i + 1]), f2_splat(12582912.0f));
+    }
+}
+
+// One 32-column chunk of one output row, dequantized in packed pairs:
+//   y[j] = (row_scale * sc[j]) * acc[j] + bias[j]   (+ GeLU),
+// one fused multiply-add per value after the exact int32 -> fp32 conversion.
+// UNI: all 32 columns share one scale (sc[0]).  Bias from shared memory
+// (bias_s) or, when bias_s is null, from global memory through L1 (bias_g,
+// 16-byte loads; columns at or past nb read 0; bias_g may then be null).
+template <bool GELU, bool UNI>
+__device__ __forceinline__ void dequant_chunk(uint32_t (&v)[32], float row_scale, const float* sc,
+                                              const float* bias_s, const float* bias_g, int nb,
+                                              uint64_t (&f)[16]) {
+    acc32_to_f2(v, f);
+    const uint64_t rs2 = f2_splat(row_scale);
+    const uint64_t a_uni = f2_splat(row_scale * sc[0]);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        uint64_t b01, b23;
+        if (bias_s) {
+            b01 = *reinterpret_cast<const uint64_t*>(bias_s + 4 * q);
+            b23 = *reinterpret_cast<const uint64_t*>(bias_s + 4 * q + 2);
+        } else {
+            const float4 t4 = 4 * q < nb ? __ldg(reinterpret_cast<const float4*>(bias_g) + q)
+                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+            b01 = f2_pack(t4.x, t4.y);
+            b23 = f2_pack(t4.z, t4.w);
+        }
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int i = 2 * q + e;
+            const uint64_t a2 = UNI ? a_uni : f2_mul(rs2, *reinterpret_cast<const uint64_t*>(sc + 2 * i));
+            uint64_t t = f2_fma(a2, f[i], e ? b23 : b01);
+            if (GELU) t = gelu2(t);
+            f[i] = t;
+        }
+    }
+}
+
+// The same with the column factors held across the warp: lane l carries the
+// weight-group scale (ca) and the bias (cb, 0 without bias) of column l of the
+// chunk; they reach every lane by shuffles (no shared-memory staging).
+template <bool GELU, bool UNI>
+__device__ __forceinline__ void dequant_chunk_lanes(uint32_t (&v)[32], float row_scale, float ca, float cb,
+                                                    uint64_t (&f)[16]) {
+    acc32_to_f2(v, f);
+    const uint64_t rs2 = f2_splat(row_scale);
+    const uint64_t a_uni = f2_splat(row_scale * __shfl_sync(0xFFFFFFFFu, ca, 0));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const uint64_t a2 = UNI ? a_uni
+                                : f2_mul(rs2, f2_pack(__shfl_sync(0xFFFFFFFFu, ca, 2 * i),
+                                                      __shfl_sync(0xFFFFFFFFu, ca, 2 * i + 1)));
+        const uint64_t b2 = f2_pack(__shfl_sync(0xFFFFFFFFu, cb, 2 * i), __shfl_sync(0xFFFFFFFFu, cb, 2 * i + 1));
+        uint64_t t = f2_fma(a2, f[i], b2);
+        if (GELU) t = gelu2(t);
+        f[i] = t;
+    }
+}
+
 // Codes of four fp32 values packed little-endian into one word.
 // t = fl(y * inv) as a packed multiply; then fl(t + 1.5*2^23) (a scalar add
 // with explicit round-to-nearest, which is never contracted with the multiply)
