@@ -240,32 +240,34 @@ w8a8_requant_cluster_kernel(const __grid_constant__ CUtensorMap tmA,
         uint8_t* stg0 = gbase + (sStg - base) + (uint32_t)(warp - 2) * NSTG * 32u * 32u;  // this warp's boxes
         const bool gelu = p.act == ZQ_ACT_GELU;
         const bool uni = p.G % CW == 0;  // every 32-column chunk lies in one weight group
+        // This CTA's columns are the same for every row block: stage their
+        // weight-group scales and biases once.
+        for (int i = et; i < 2 * BN; i += kEpiThreads) {
+            const int h = i / BN, c = i % BN;
+            const int n = (2 * rank + h) * BN + c;
+            const bool in = n < p.N;
+            col_f[h * 2 * BN + c] = in ? __ldg(p.s_grp + n / p.G) : 0.0f;
+            col_f[h * 2 * BN + BN + c] = (in && p.bias) ? __ldg(p.bias + n) : 0.0f;
+        }
+        named_bar_sync(1, kEpiThreads);
+        float next_scale = (cl < m_tiles && cl * BM + r < p.M) ? __ldg(p.s_tok + cl * BM + r) : 0.0f;
         uint32_t mbi = 0;
-        bool alive = true;
-        for (int mb = cl; alive && mb < m_tiles; mb += ncl, ++mbi) {
-            // column factors of both halves (previous readers are done)
-            named_bar_sync(1, kEpiThreads);
-            for (int i = et; i < 2 * BN; i += kEpiThreads) {
-                const int h = i / BN, c = i % BN;
-                const int n = (2 * rank + h) * BN + c;
-                const bool in = n < p.N;
-                col_f[h * 2 * BN + c] = in ? __ldg(p.s_grp + n / p.G) : 0.0f;
-                col_f[h * 2 * BN + BN + c] = (in && p.bias) ? __ldg(p.bias + n) : 0.0f;
-            }
-            named_bar_sync(1, kEpiThreads);
+        for (int mb = cl; mb < m_tiles; mb += ncl, ++mbi) {
             const int gm = mb * BM + r;
             const bool row_ok = gm < p.M;
-            const float row_scale = row_ok ? __ldg(p.s_tok + gm) : 0.0f;
+            const float row_scale = next_scale;  // loaded one row block ahead
+            const int gn = gm + ncl * BM;
+            next_scale = (mb + ncl < m_tiles && gn < p.M) ? __ldg(p.s_tok + gn) : 0.0f;
 
-            // pass 1: y = dequant + bias (+GeLU); written back to TMEM; partial absmax
+            // pass 1: y = dequant + bias (+GeLU); written back to TMEM; partial
+            // absmax.  Warps go at their own pace; a failed wait is carried to the
+            // exchange barrier below, where all epilogue threads agree on it.
             float pmax = 0.0f;
-            for (int h = 0; h < 2; ++h) {
+            bool ok = true;
+            for (int h = 0; ok && h < 2; ++h) {
                 if (!(h ? real1 : real0)) continue;
-                const bool got = mbar_wait(bar_tfull(h), mbi & 1u, abort_flag, p.status, SITE_E_TFULL);
-                if (!named_bar_and(1, kEpiThreads, got)) {
-                    alive = false;
-                    break;
-                }
+                ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar_tfull(h), mbi & 1u, abort_flag, p.status, SITE_E_TFULL));
+                if (!ok) break;
                 tc_fence_after();
                 const float* sc = col_f + h * 2 * BN;
                 const float* bi = sc + BN;
@@ -288,7 +290,6 @@ w8a8_requant_cluster_kernel(const __grid_constant__ CUtensorMap tmA,
                 }
                 tmem_st_wait();
             }
-            if (!alive) break;
 
             // exchange: row absmax over this CTA's column slices, then over the cluster
             // Each CTA's exchange barrier expects C * BM * 4 bytes per use; every
@@ -299,8 +300,8 @@ w8a8_requant_cluster_kernel(const __grid_constant__ CUtensorMap tmA,
             // which needs every CTA's next-block partials, sent after reading.
             const int buf = mbi & 1;
             slice_part[slice * BM + r] = pmax;
-            if (et == 0) mbar_arrive_expect_tx(bar_xchg(buf), (uint32_t)(p.C * BM * 4));
-            named_bar_sync(1, kEpiThreads);
+            if (et == 0 && ok) mbar_arrive_expect_tx(bar_xchg(buf), (uint32_t)(p.C * BM * 4));
+            if (!named_bar_and(1, kEpiThreads, ok)) break;
             if (slice == 0) {
                 float m = slice_part[r];
 #pragma unroll
