@@ -68,6 +68,12 @@ class L2Flush:
         self.sink.copy_(self.buf.max().view(1))
 
 
+def ridge_ops_per_byte():
+    """Ops per byte where the int8 tensor peak meets HBM bandwidth."""
+    pk = load_peaks()
+    return INT8_OVER_BF16 * pk["bf16_tflops"] * 1e12 / (pk["hbm_gbs"] * 1e9)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -257,7 +263,16 @@ def build_workload(name, zq, torch, device):
         Kd = Wq.shape[1]
         ops = 2 * T * N * Kd
         W.ops += ops
-        W.kernel_units[label] = ("tensor", ops, "ops")
+        # algorithmic bytes: activations and weights in once, outputs out once
+        out_b = T * N * (1 if out_kind == zq.ZQ_OUT_I8_REQUANT else y.element_size()) + \
+            (4 * T if out_kind == zq.ZQ_OUT_I8_REQUANT else 0)
+        lin_bytes = T * Kd + 4 * T + N * Kd + 4 * (N // G) + (4 * N if b is not None else 0) + out_b
+        # the roofline that binds: HBM when the ops per byte fall below the
+        # ridge point (int8 peak / HBM bandwidth), the tensor cores otherwise
+        if ops / lin_bytes < ridge_ops_per_byte():
+            W.kernel_units[label] = ("hbm", lin_bytes, "bytes")
+        else:
+            W.kernel_units[label] = ("tensor", ops, "ops")
         a_q, a_s = y, s_out
         W.out = y
     W.config.update(layers=[list(l[0].shape) + [l[3]] for l in layers],
@@ -516,7 +531,8 @@ def main(argv=None):
                 "traffic": recorded_traffic(a.workload, dom), "stage_ms": round(stage_ms[dom], 5)}
     else:
         achieved = units / (stage_ms[dom] * 1e-3) / 1e9
-        roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
+        roof = {"kernel": dom if dom.endswith("quant") else f"w8a8 linear ({dom})", "bound": "hbm",
+                "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "peak_source": f"{peaks['source']} copy bandwidth",
                 "frac_vs_spec": round(achieved / SPEC_HBM_GBS, 4),

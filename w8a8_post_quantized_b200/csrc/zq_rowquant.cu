@@ -217,6 +217,22 @@ rowq_pipe_kernel(const Tin* __restrict__ x, int T, int H, float inv_h, int R, in
     }
     griddep_wait();  // inputs and outputs are free of the previous grid in the stream
     griddep_launch_dependents();
+
+    auto issue = [&](int u, int s) {
+        const int rows = min(R, T - u * R);
+        const uint32_t bytes = (uint32_t)(rows * row_bytes);
+        mbar_arrive_expect_tx(bar0 + 8u * s, bytes);
+        bulk_load(smem_u32(ring + (size_t)s * stage_bytes), x + (int64_t)u * R * H, bytes, bar0 + 8u * s);
+    };
+    // the first row blocks are requested before the parameters are staged, so
+    // the two global-memory latencies overlap (the ring lies past the
+    // parameter area; the other threads wait on the barriers only after the
+    // __syncthreads below, which also publishes their initialisation)
+    if (threadIdx.x == 0)
+        for (int j = 0; j < nstages; ++j) {
+            const int u = blockIdx.x + j * gridDim.x;
+            if (u < n_units) issue(u, j);
+        }
     if constexpr (SMEMP) {
         const float* src0 = LN ? gamma : bias;
         constexpr int QPP = NP / 2;  // 16-byte quarters per piece
@@ -230,18 +246,6 @@ rowq_pipe_kernel(const Tin* __restrict__ x, int T, int H, float inv_h, int R, in
     const float* pb = SMEMP ? spar + H : beta;
     const float* pbias = SMEMP ? spar : bias;
     __syncthreads();
-
-    auto issue = [&](int u, int s) {
-        const int rows = min(R, T - u * R);
-        const uint32_t bytes = (uint32_t)(rows * row_bytes);
-        mbar_arrive_expect_tx(bar0 + 8u * s, bytes);
-        bulk_load(smem_u32(ring + (size_t)s * stage_bytes), x + (int64_t)u * R * H, bytes, bar0 + 8u * s);
-    };
-    if (threadIdx.x == 0)
-        for (int j = 0; j < nstages; ++j) {
-            const int u = blockIdx.x + j * gridDim.x;
-            if (u < n_units) issue(u, j);
-        }
 
     int j = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++j) {
