@@ -211,11 +211,14 @@ __device__ __forceinline__ uint64_t u2_pack(uint32_t lo, uint32_t hi) {
 
 // GeLU of a pair of values in packed fp32 arithmetic, the approximation of
 // gelu_f rearranged to need no select: with a = |x| and L = Phi(-a),
-//   gelu(x) = x * Phi(x) = max(x, 0) - a * L
-// (x >= 0: x - x L;  x < 0: x * Phi(x) = x * Phi(-a) = -a L).  L is the
-// Abramowitz & Stegun 7.1.26 form t P(t) exp(-a^2/2) / 2, t = 1/(1 + p a/sqrt2);
-// the coefficients enter negated and halved so that the last step is one
-// fused multiply-add: gelu = max(x, 0) + (t Q(t) a) exp(-a^2/2), Q = -P/2.
+//   gelu(x) = x * Phi(x) = x/2 + a * (1/2 - L)
+// (x >= 0: x/2 + x/2 - x L = x - x L;  x < 0: x/2 - x/2 + x L = x Phi(x)).  L is
+// the Abramowitz & Stegun 7.1.26 form t P(t) exp(-a^2/2) / 2 with
+// t = 1/(1 + p a/sqrt2); the coefficients enter negated and halved (Q = -P/2)
+// so that 1/2 - L = fma(t Q(t), exp(-a^2/2), 1/2) and the last step is one
+// fused multiply-add.  For x < 0 the two halves cancel inside that FMA, which
+// leaves an absolute error of about |x| 2^-25 (far below the approximation's
+// 1.5e-7 * |x|).
 __device__ __forceinline__ uint64_t gelu2(uint64_t x2) {
     constexpr float kPs = 0.3275911f * 0.70710678118654752f;
     constexpr float kB1 = -0.5f * 0.254829592f, kB2 = -0.5f * -0.284496736f, kB3 = -0.5f * 1.421413741f,
@@ -235,39 +238,18 @@ __device__ __forceinline__ uint64_t gelu2(uint64_t x2) {
     h = f2_fma(t2, h, f2_splat(kB3));
     h = f2_fma(t2, h, f2_splat(kB2));
     h = f2_fma(t2, h, f2_splat(kB1));
-    const uint64_t ta = f2_mul(t2, a2);
-    return f2_fma(f2_mul(h, ta), f2_pack(e0, e1), f2_pack(fmaxf(x0, 0.0f), fmaxf(x1, 0.0f)));
+    const uint64_t w = f2_fma(f2_mul(h, t2), f2_pack(e0, e1), f2_splat(0.5f));  // 1/2 - L
+    return f2_fma(a2, w, f2_mul(x2, f2_splat(0.5f)));
 }
 
-// Exact int32 -> fp32 of a pair without the conversion unit, for |v| < 2^22:
-// the word 0x4B400000 + v is the float 1.5*2^23 + v, and subtracting 1.5*2^23
-// is exact.  `bad` accumulates a word whose bits 23..31 are all zero exactly
-// when every converted v was in range (0x4B400000 + v within [2^23, 2^24)).
-__device__ __forceinline__ uint64_t i2f2_magic(uint32_t v0, uint32_t v1, uint32_t& bad) {
-    const uint32_t w0 = v0 + 0x4B400000u, w1 = v1 + 0x4B400000u;
-    bad |= (w0 ^ 0x4B000000u) | (w1 ^ 0x4B000000u);
-    return f2_sub(u2_pack(w0, w1), f2_splat(12582912.0f));
-}
-constexpr uint32_t kI2fBadMask = 0xFF800000u;
-
-// 32 int32 accumulators -> 16 packed fp32 pairs, exact: the conversion-unit
-// free path when every |acc| < 2^22, else the hardware conversion.  `v` is
-// modified (offset words) on return.
-__device__ __forceinline__ void acc32_to_f2(uint32_t (&v)[32], uint64_t (&f)[16]) {
-    uint32_t bad = 0;
+// 32 int32 accumulators -> 16 packed fp32 pairs, rounded to nearest (exact
+// while |acc| < 2^24, which holds for any K <= 1040).  A variant that avoids
+// cvt -- the word 0x4B400000 + acc read as the float 1.5*2^23 + acc, with a
+// per-chunk range check -- measured slower on B200: the check costs more
+// issue slots than the conversion.
+__device__ __forceinline__ void acc32_to_f2(const uint32_t (&v)[32], uint64_t (&f)[16]) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-        v[j] += 0x4B400000u;  // 1.5*2^23 + acc as a float, when |acc| < 2^22
-        bad |= v[j] ^ 0x4B000000u;
-    }
-    if (bad & kI2fBadMask) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-            f[i] = f2_pack((float)(int)(v[2 * i] - 0x4B400000u), (float)(int)(v[2 * i + 1] - 0x4B400000u));
-    } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) f[i] = f2_sub(u2_pack(v[2 * i], v[2 * i + 1]), f2_splat(12582912.0f));
-    }
+    for (int i = 0; i < 16; ++i) f[i] = f2_pack((float)(int)v[2 * i], (float)(int)v[2 * i + 1]);
 }
 
 // One 32-column chunk of one output row, dequantized in packed pairs:
