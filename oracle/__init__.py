@@ -14,6 +14,8 @@ Sources (web pages):
   [TS36] "探秘Transformer系列之（36）— 大模型量化方案" -- §1.1.2, §1.2.2.
   [IQ]   "Integer Quantization: Deep Dive" -- quantization formula,
          fake quantization, quantization error.
+  [SQ]   "SmoothQuant技术解析：大模型INT8量化的突破与实践" §2.2, §3 and [TS36]
+         §1.3 -- per-channel smoothing folded offline into the weights.
 
 Every function here is pinned by ``tests/test_oracle_pins.py`` against
 hand-worked examples (``tests/golden/``), closed forms, invariants and
@@ -64,6 +66,10 @@ def _L():
             "zqo_bias_act": [P, I64, I64, P, ctypes.c_int, P],
             "zqo_gemm_i32": [P, I64, I64, P, I64, P],
             "zqo_dequant": [P, I64, I64, P, P, I64, P, ctypes.c_int, P],
+            "zqo_channel_absmax": [P, I64, I64, P],
+            "zqo_weight_col_absmax": [P, I64, I64, P],
+            "zqo_smooth_factors": [P, P, I64, ctypes.c_double, P],
+            "zqo_smooth_fold": [P, I64, I64, P, P, P, P, P, P],
         }
         for name, args in sig.items():
             fn = getattr(lib, name)
@@ -172,6 +178,53 @@ def dequant(acc, s_tok, s_grp, group_rows, bias=None, act=ACT_NONE):
     return y
 
 
+def channel_absmax(a, amax=None):
+    """Running per-channel absmax of an activation a [T, H] ([SQ] §3 calibration)."""
+    a, pa = _c(a, np.float32)
+    T, H = a.shape
+    out = np.zeros(H, np.float32) if amax is None else np.array(amax, np.float32, copy=True)
+    _chk(_L().zqo_channel_absmax(pa, T, H, out.ctypes.data), "channel_absmax")
+    return out
+
+
+def weight_col_absmax(W):
+    """Per input channel absmax of W [N, K]: max over the N output rows."""
+    W, pw = _c(W, np.float32)
+    N, K = W.shape
+    out = np.empty(K, np.float32)
+    _chk(_L().zqo_weight_col_absmax(pw, N, K, out.ctypes.data), "weight_col_absmax")
+    return out
+
+
+def smooth_factors(amax, wmax, alpha=0.5):
+    """s_j = amax_j^alpha / wmax_j^(1-alpha) (reading R9 of zq_oracle.c)."""
+    a, pa = _c(amax, np.float32)
+    w, pw = _c(wmax, np.float32)
+    s = np.empty(a.size, np.float32)
+    _chk(_L().zqo_smooth_factors(pa, pw, a.size, float(alpha), s.ctypes.data), "smooth_factors")
+    return s
+
+
+def smooth_fold(W, s, gamma=None, beta=None):
+    """W' = W diag(s) per input channel; gamma' = gamma / s, beta' = beta / s."""
+    W, pw = _c(W, np.float32)
+    s_, ps = _c(s, np.float32)
+    N, K = W.shape
+    Wo = np.empty((N, K), np.float32)
+    pg = pb = None
+    go = bo = None
+    if gamma is not None:
+        gamma, pg = _c(gamma, np.float32)
+        go = np.empty(K, np.float32)
+    if beta is not None:
+        beta, pb = _c(beta, np.float32)
+        bo = np.empty(K, np.float32)
+    _chk(_L().zqo_smooth_fold(pw, N, K, pg, pb, ps, Wo.ctypes.data,
+                              None if go is None else go.ctypes.data,
+                              None if bo is None else bo.ctypes.data), "smooth_fold")
+    return Wo, go, bo
+
+
 # ---- compositions, in the order of the fused flowcharts of [ZQ] ----------
 
 def ln_quant(x, gamma, beta, eps):
@@ -202,3 +255,16 @@ def ffn_block(x, gamma, beta, eps, W1q, s1, b1, W2q, s2, b2, group_rows):
     q2, st2 = linear_requant(q1, st1, W1q, s1, group_rows, b1, ACT_GELU)
     y = linear(q2, st2, W2q, s2, group_rows, b2, ACT_NONE)
     return y, (q1, st1, q2, st2)
+
+
+def smooth_ln_linear(calib_batches, gamma, beta, eps, W, alpha=0.5):
+    """SmoothQuant offline step for a linear fed by a LayerNorm ([TS36] §1.3,
+    [SQ] §3): calibrate the per-channel absmax of the LayerNorm output over
+    the batches, derive s, fold diag(s)^-1 into gamma/beta and diag(s) into
+    W.  Returns (W', gamma', beta', s, activation absmax)."""
+    amax = None
+    for xb in calib_batches:
+        amax = channel_absmax(layernorm(xb, gamma, beta, eps), amax)
+    s = smooth_factors(amax, weight_col_absmax(W), alpha)
+    Wo, go, bo = smooth_fold(W, s, gamma, beta)
+    return Wo, go, bo, s, amax

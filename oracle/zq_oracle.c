@@ -27,6 +27,13 @@
  *          with scale, zero-point, round-to-nearest and clamp); "量化模拟"
  *          (dequantize x = s * (x_int - z)); "量化误差" (rounding error is
  *          at most s/2).
+ *   [TS36] §1.3 SmoothQuant -- per-channel smoothing factor s chosen
+ *          offline; Y = (X diag(s)^-1)(diag(s) W): weights scaled up per
+ *          input channel, activations scaled down, output unchanged.
+ *   [SQ]   "SmoothQuant技术解析：大模型INT8量化的突破与实践" §2.2 (the same
+ *          identity; s chosen so the channels of X diag(s)^-1 have similar
+ *          absolute maxima), §3 (calibration of per-channel max |X| over
+ *          calibration batches; offline fold into the weights).
  *
  * Readings where the pages are silent (each one is a choice, stated once):
  *   R1 round-to-nearest ties go to even (rintf under the default mode);
@@ -38,6 +45,15 @@
  *   R6 LayerNorm uses the biased variance with eps inside the square root;
  *   R7 GeLU is the exact erf form 0.5 x (1 + erf(x / sqrt 2));
  *   R8 bias is added after dequantization, in floating point.
+ *   R9 the smoothing factor is the SmoothQuant paper's balance rule (the
+ *      pages name the paper but are cut off before its formula):
+ *      s_j = amax_x[j]^alpha / amax_w[j]^(1 - alpha), alpha the migration
+ *      strength (0.5 balances both maxima; 1 equalises the activation
+ *      channels); computed in double, rounded to fp32, at least 1e-5; a
+ *      channel whose activation or weight absmax is 0 keeps s_j = 1;
+ *  R10 the activation diag(s)^-1 is folded into the preceding LayerNorm's
+ *      gamma and beta (the normalised row is divided per channel), so the
+ *      online path is unchanged.
  *
  * Status codes: 0 = ok, 1 = bad argument, 2 = int32 overflow in the GEMM.
  */
@@ -186,5 +202,66 @@ int zqo_dequant(const int32_t* acc, int64_t T, int64_t N, const float* s_tok,
             if (act == 1) v = gelu_d(v);
             y[t * N + o] = (float)v;
         }
+    return ZQO_OK;
+}
+
+/* [SQ] §3 calibration: running per-channel absmax of an activation a [T, H]
+ * (the input of the linear): amax[j] = max(amax[j], max_t |a[t, j]|).
+ * Max is exact, so no rounding enters. */
+int zqo_channel_absmax(const float* a, int64_t T, int64_t H, float* amax)
+{
+    if (!a || !amax || T <= 0 || H <= 0) return ZQO_EARG;
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t j = 0; j < H; ++j) {
+            float v = fabsf(a[t * H + j]);
+            if (v > amax[j]) amax[j] = v;
+        }
+    return ZQO_OK;
+}
+
+/* Per input channel (column j of W [N, K]) absmax: wmax[j] = max_o |W[o, j]|. */
+int zqo_weight_col_absmax(const float* W, int64_t N, int64_t K, float* wmax)
+{
+    if (!W || !wmax || N <= 0 || K <= 0) return ZQO_EARG;
+    for (int64_t j = 0; j < K; ++j) wmax[j] = 0.0f;
+    for (int64_t o = 0; o < N; ++o)
+        for (int64_t j = 0; j < K; ++j) {
+            float v = fabsf(W[o * K + j]);
+            if (v > wmax[j]) wmax[j] = v;
+        }
+    return ZQO_OK;
+}
+
+/* [TS36] §1.3 / [SQ] §2.2, reading R9: s_j = amax_j^alpha / wmax_j^(1-alpha). */
+int zqo_smooth_factors(const float* amax, const float* wmax, int64_t K, double alpha, float* s)
+{
+    if (!amax || !wmax || !s || K <= 0 || !(alpha >= 0.0 && alpha <= 1.0)) return ZQO_EARG;
+    for (int64_t j = 0; j < K; ++j) {
+        if (amax[j] == 0.0f || wmax[j] == 0.0f) {
+            s[j] = 1.0f;
+            continue;
+        }
+        double v = pow((double)amax[j], alpha) / pow((double)wmax[j], 1.0 - alpha);
+        float f = (float)v;
+        s[j] = f < 1e-5f ? 1e-5f : f;
+    }
+    return ZQO_OK;
+}
+
+/* [TS36] §1.3 identity, reading R10: W_out[o, j] = W[o, j] * s_j (each
+ * output row scaled per input channel), gamma_out[j] = gamma[j] / s_j,
+ * beta_out[j] = beta[j] / s_j; each computed in double and rounded once to
+ * fp32 (gamma or beta may be NULL: not folded). */
+int zqo_smooth_fold(const float* W, int64_t N, int64_t K, const float* gamma, const float* beta,
+                    const float* s, float* W_out, float* gamma_out, float* beta_out)
+{
+    if (!W || !s || !W_out || N <= 0 || K <= 0) return ZQO_EARG;
+    if ((gamma && !gamma_out) || (beta && !beta_out)) return ZQO_EARG;
+    for (int64_t o = 0; o < N; ++o)
+        for (int64_t j = 0; j < K; ++j) W_out[o * K + j] = (float)((double)W[o * K + j] * (double)s[j]);
+    for (int64_t j = 0; j < K; ++j) {
+        if (gamma) gamma_out[j] = (float)((double)gamma[j] / (double)s[j]);
+        if (beta) beta_out[j] = (float)((double)beta[j] / (double)s[j]);
+    }
     return ZQO_OK;
 }
