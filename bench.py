@@ -184,6 +184,8 @@ class Workload:
         self.h2d = None           # (pinned host tensor, device tensor) of the step's input
         self.d2h = None           # (device tensor, pinned host tensor) of the step's result
         self.kernel_units = {}    # stage label -> (bound, algorithmic units per launch, unit)
+        self.bytes = 0            # algorithmic bytes per step when the metric is bandwidth
+        self.metric = None
         self.config = {}
 
     def dev(self, a):
@@ -195,8 +197,43 @@ class Workload:
         return self.dev(a.f32)
 
 
+def build_smooth_workload(W, zq, torch, device):
+    """SmoothQuant offline steps on the BERT-base FFN's first linear: the
+    calibration pass over the LayerNorm output of the 4096-token batch and
+    the factor + fold of W1 [3072, 768] (and gamma, beta).  HBM-bound."""
+    w = inputs.bert_ffn()
+    lin = w.layers[0]
+    x = W.dev_act(w.x)
+    T, H = x.shape
+    g, b = W.dev(w.gamma), W.dev(w.beta)
+    W1 = W.dev(lin.W)
+    N = W1.shape[0]
+    amax = torch.zeros(H, dtype=torch.float32, device=device)
+    W1o, go, bo = torch.empty_like(W1), torch.empty_like(g), torch.empty_like(b)
+    sf = torch.empty(H, dtype=torch.float32, device=device)
+    # the calibration is a running max: repeating it on the same batch is idempotent
+    W.stages.append(("smooth_calibrate", lambda: zq.zq_smooth_calibrate(x, g, b, w.eps, amax=amax)))
+    W.stages.append(("smooth_weights", lambda: zq.zq_smooth_weights(W1, amax, 0.5, g, b, W_out=W1o,
+                                                                     gamma_out=go, beta_out=bo, s=sf)))
+    xbytes = x.numel() * x.element_size()
+    # algorithmic bytes: x, gamma, beta read once, amax read and written;
+    # W read once and W' written once, plus the per-channel vectors
+    W.kernel_units["smooth_calibrate"] = ("hbm", xbytes + 8 * H + 8 * H, "bytes")
+    W.kernel_units["smooth_weights"] = ("hbm", 8 * N * H + 6 * 4 * H, "bytes")
+    W.bytes = sum(v[1] for v in W.kernel_units.values())
+    W.metric = "SmoothQuant calibration + weight fold GB/s (algorithmic bytes)"
+    W.tokens = T
+    W.h2d_src = x
+    W.out = sf
+    W.config = {"workload": "bert_ffn W1 SmoothQuant (calibrate LN output 4096x768 bf16, fold W1 3072x768)",
+                "tokens": T, "hidden": H, "x_dtype": w.x.dtype, "alpha": 0.5}
+    return W
+
+
 def build_workload(name, zq, torch, device):
     W = Workload(name, zq, torch, device)
+    if name == "bert_smooth":
+        return build_smooth_workload(W, zq, torch, device)
     if name in ("bert_ffn", "gptj_qkv", "tiny"):
         w = {"bert_ffn": inputs.bert_ffn, "gptj_qkv": inputs.gptj_qkv, "tiny": inputs.tiny}[name]()
     elif name == "neox_decode":
@@ -441,6 +478,8 @@ def oracle_sample(name, budget_s=12.0, max_rows=None):
     elif name.startswith("gemm_sweep_"):
         M = int(name.split("_")[-1])
         w = inputs.gemm_sweep_point(M, inputs.GEMM_SWEEP_M.index(M))
+    elif name == "bert_smooth":
+        return oracle_smooth_sample(budget_s, max_rows)
     else:
         raise SystemExit(f"no oracle baseline for {name}")
     qlayers = [(*oracle.quantize_weights(l.W, l.group_rows), l.bias, l.group_rows) for l in w.layers]
@@ -466,6 +505,34 @@ def oracle_sample(name, budget_s=12.0, max_rows=None):
         t_total += time.perf_counter() - t0
         rows_done += x.shape[0]
     return ops, t_total, rows_done, T
+
+
+def oracle_smooth_sample(budget_s=12.0, max_rows=None):
+    """The oracle's SmoothQuant steps on a bounded sample: the calibration of
+    a row sample of the BERT batch, then the factors and fold of all of W1.
+    Returns (algorithmic bytes done, seconds, rows, total rows)."""
+    import oracle
+    w = inputs.bert_ffn()
+    lin = w.layers[0]
+    T, H = w.x.f32.shape
+    N = lin.W.shape[0]
+    e = 2 if w.x.dtype == "bf16" else 4
+    rows_done, nbytes, t_total = 0, 0, 0.0
+    limit = max_rows if max_rows is not None else T
+    amax = None
+    while rows_done < limit and t_total < budget_s * 0.5:
+        x = w.x.f32[rows_done % T:rows_done % T + 8]
+        t0 = time.perf_counter()
+        amax = oracle.channel_absmax(oracle.layernorm(x, w.gamma, w.beta, w.eps), amax)
+        t_total += time.perf_counter() - t0
+        rows_done += x.shape[0]
+        nbytes += x.shape[0] * H * e
+    t0 = time.perf_counter()
+    s = oracle.smooth_factors(amax, oracle.weight_col_absmax(lin.W), 0.5)
+    oracle.smooth_fold(lin.W, s, w.gamma, w.beta)
+    t_total += time.perf_counter() - t0
+    nbytes += 8 * N * H + 16 * H
+    return nbytes, t_total, rows_done, T
 
 
 # -------------------------------------------------------------------- main
@@ -537,31 +604,33 @@ def main(argv=None):
                 "peak_source": f"{peaks['source']} copy bandwidth",
                 "frac_vs_spec": round(achieved / SPEC_HBM_GBS, 4),
                 "traffic": recorded_traffic(a.workload, dom), "stage_ms": round(stage_ms[dom], 5)}
-    qlabel = "ln_quant" if "ln_quant" in stage_ms else "act_quant"
-    qb = W.kernel_units[qlabel][1]
-    q_gbs = qb / (stage_ms[qlabel] * 1e-3) / 1e9
+    qlabel = "ln_quant" if "ln_quant" in stage_ms else ("act_quant" if "act_quant" in stage_ms else None)
+    qb = W.kernel_units[qlabel][1] if qlabel else 0
+    q_gbs = qb / (stage_ms[qlabel] * 1e-3) / 1e9 if qlabel else None
 
     if W.ops:
         metric, unit = "W8A8 linear INT8 TOPS (whole step, incl. fused LN/token-quant)", "TOPS"
         value = world * W.ops / (ms_per_step * 1e-3) / 1e12
         e2e_value = world * W.ops / (e2e_ms * 1e-3) / 1e12
     else:
-        metric, unit = "fused LN/token-quant GB/s", "GB/s"
-        value = world * qb / (ms_per_step * 1e-3) / 1e9
-        e2e_value = world * qb / (e2e_ms * 1e-3) / 1e9
+        metric, unit = W.metric or "fused LN/token-quant GB/s", "GB/s"
+        step_bytes = W.bytes or qb
+        value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
+        e2e_value = world * step_bytes / (e2e_ms * 1e-3) / 1e9
 
     out = {
         "metric": metric, "value": round(value, 2), "unit": unit, "n_gpus": world,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms_per_step, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8" if W.ops or W.metric is None else "f32",
         "data": "synthetic (seeded; layer shapes only, random weights)",
         "config": dict(W.config, parallelism=f"replicas x{world}",
                        l2="flushed before every timed step (256 MiB write + read-back)",
                        timing="one CUDA graph per step (kernels chained by programmatic dependent launch), CUDA events on the launching stream; per-stage times from per-stage graphs"),
         "tokens_per_s": round(world * W.tokens / (ms_per_step * 1e-3), 1),
         "stages_ms": {k: round(v, 5) for k, v in stage_ms.items()},
-        "ln_quant_gbs": round(q_gbs, 1),
-        "ln_quant_frac_hbm": round(q_gbs / peaks["hbm_gbs"], 4),
+        "ln_quant_gbs": round(q_gbs, 1) if q_gbs else None,
+        "ln_quant_frac_hbm": round(q_gbs / peaks["hbm_gbs"], 4) if q_gbs else None,
         "roofline": roof,
         "e2e": {"value": round(e2e_value, 3), "unit": unit, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
@@ -596,17 +665,22 @@ def main_reference(a, rank, world):
             ops_tot += ops
             secs_tot += secs
             rows_tot += rows
-    value = ops_tot / secs_tot / 1e12
-    metric = "W8A8 linear INT8 TOPS (whole step, incl. fused LN/token-quant)"
-    out = {"impl": "reference", "metric": metric, "value": round(value, 8), "unit": "TOPS",
+    if a.workload == "bert_smooth":
+        value = ops_tot / secs_tot / 1e9
+        metric, unit = "SmoothQuant calibration + weight fold GB/s (algorithmic bytes)", "GB/s"
+    else:
+        value = ops_tot / secs_tot / 1e12
+        metric, unit = "W8A8 linear INT8 TOPS (whole step, incl. fused LN/token-quant)", "TOPS"
+    out = {"impl": "reference", "metric": metric, "value": round(value, 8), "unit": unit,
            "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
            "ms_per_step": round(1e3 * secs_tot / a.steps, 3), "higher_is_better": True,
-           "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+           "scaling": "weak", "vs_baseline": None, "dtype": "f32" if a.workload == "bert_smooth" else "int8",
+           "data": "synthetic",
            "config": {"workload": a.workload, "sample_rows_per_step": rows_tot // max(1, a.steps),
                       "total_rows": T},
-           "cpu_baseline": {"value": round(value, 8), "unit": "TOPS", "cores": 1, "kind": "oracle",
+           "cpu_baseline": {"value": round(value, 8), "unit": unit, "cores": 1, "kind": "oracle",
                             "sample": f"{rows_tot // max(1, a.steps)} token rows per step of {T}"},
-           "e2e": {"value": round(value, 8), "unit": "TOPS", "h2d_bytes_per_step": 0,
+           "e2e": {"value": round(value, 8), "unit": unit, "h2d_bytes_per_step": 0,
                    "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
     return 0

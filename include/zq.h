@@ -198,6 +198,50 @@ int zq_w8a8_linear_requant_noalloc(const int8_t* xq, const float* s_tok, int64_t
                                    int64_t group_rows, const float* bias, int act,
                                    int8_t* y, float* s_tok_out, void* stream);
 
+/* ---- SmoothQuant smoothing (offline) ------------------------------------
+ * [TS36] §1.3 SmoothQuant; "SmoothQuant技术解析：大模型INT8量化的突破与实践"
+ * §2.2, §3.  Y = (X diag(s)^-1)(diag(s) W) is the same output; a per-channel
+ * s chosen offline makes the activation channels' maxima alike, so per-token
+ * activation quantization loses less to outlier channels.  The activation
+ * side is folded into the LayerNorm feeding the linear, so the online calls
+ * (zq_ln_quant, zq_w8a8_linear) run unchanged on the smoothed parameters.
+ *
+ * zq_smooth_calibrate: running per-channel absmax of the linear's input over
+ * calibration batches.  The activation is a = LayerNorm(x; gamma, beta, eps)
+ * (as zq_ln_quant computes it, beta may be NULL for 0) when gamma is
+ * non-NULL, else a = x.  amax[j] = max(amax[j], max_t |a[t, j]|).
+ * x      : [T, H] device, dtype x_dtype (ZQ_F32 or ZQ_BF16).
+ * amax   : fp32 [H] device, in/out; fill it with zeros before the first
+ *          batch; it must hold values >= 0.
+ * Constraints: H % 16 == 0, H <= 32768.  Errors: NULL, SHAPE, ALIGN,
+ * DTYPE, CUDA, DEVICE. */
+int zq_smooth_calibrate(const void* x, int x_dtype, int64_t T, int64_t H,
+                        const float* gamma, const float* beta, float eps,
+                        float* amax, void* stream);
+
+/* zq_smooth_weights: the factors and the fold.
+ *   wmax_j = max_o |W[o, j]|;
+ *   s_j    = amax_j^alpha / wmax_j^(1 - alpha), at least 1e-5 (powers in
+ *            double, rounded once to fp32); s_j = 1 where amax_j or wmax_j
+ *            is 0 (the SmoothQuant paper's rule; the pages name the paper
+ *            but not its formula);
+ *   W_out[o, j] = W[o, j] * s_j;  gamma_out_j = gamma_j / s_j;
+ *   beta_out_j = beta_j / s_j   (each one IEEE fp32 rounding).
+ * W      : fp32 [N, K] device (output rows o, input channels j);
+ * amax   : fp32 [K] device, from zq_smooth_calibrate;
+ * alpha  : migration strength in [0, 1] (0.5 balances the activation and
+ *          weight maxima, 1 makes every activation channel's max 1);
+ * gamma, beta : fp32 [K] device or NULL (then not folded);
+ * W_out  : fp32 [N, K] device (may be W); gamma_out, beta_out : fp32 [K]
+ *          (may alias gamma, beta; required when those are given);
+ * s      : fp32 [K] device (output; also used as scratch during the call).
+ * Quantize W_out with zq_quantize_weights and pass gamma_out/beta_out to
+ * zq_ln_quant.  Constraints: K % 16 == 0.  Errors: NULL, SHAPE, ALIGN,
+ * DTYPE (alpha outside [0, 1]), CUDA, DEVICE. */
+int zq_smooth_weights(const float* W, int64_t N, int64_t K, const float* amax, float alpha,
+                      const float* gamma, const float* beta, float* W_out,
+                      float* gamma_out, float* beta_out, float* s, void* stream);
+
 /* ---- diagnostics ----------------------------------------------------------
  * zq_device_status: synchronizes `stream`, then reads and clears the device
  * flag that bounded waits set on expiry.  Returns ZQ_OK, ZQ_ERR_TIMEOUT or

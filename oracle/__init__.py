@@ -68,7 +68,7 @@ def _L():
             "zqo_dequant": [P, I64, I64, P, P, I64, P, ctypes.c_int, P],
             "zqo_channel_absmax": [P, I64, I64, P],
             "zqo_weight_col_absmax": [P, I64, I64, P],
-            "zqo_smooth_factors": [P, P, I64, ctypes.c_double, P],
+            "zqo_smooth_factors": [P, P, I64, F, P],
             "zqo_smooth_fold": [P, I64, I64, P, P, P, P, P, P],
         }
         for name, args in sig.items():
@@ -197,7 +197,8 @@ def weight_col_absmax(W):
 
 
 def smooth_factors(amax, wmax, alpha=0.5):
-    """s_j = amax_j^alpha / wmax_j^(1-alpha) (reading R9 of zq_oracle.c)."""
+    """s_j = amax_j^alpha / wmax_j^(1-alpha) (reading R9 of zq_oracle.c);
+    alpha is taken as an fp32 value, as the library's interface passes it."""
     a, pa = _c(amax, np.float32)
     w, pw = _c(wmax, np.float32)
     s = np.empty(a.size, np.float32)

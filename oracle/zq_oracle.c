@@ -232,9 +232,12 @@ int zqo_weight_col_absmax(const float* W, int64_t N, int64_t K, float* wmax)
     return ZQO_OK;
 }
 
-/* [TS36] §1.3 / [SQ] §2.2, reading R9: s_j = amax_j^alpha / wmax_j^(1-alpha). */
-int zqo_smooth_factors(const float* amax, const float* wmax, int64_t K, double alpha, float* s)
+/* [TS36] §1.3 / [SQ] §2.2, reading R9: s_j = amax_j^alpha / wmax_j^(1-alpha).
+ * alpha is an fp32 parameter (the migration strength as the library's
+ * interface passes it); the powers use its exact value in double. */
+int zqo_smooth_factors(const float* amax, const float* wmax, int64_t K, float alpha_f, float* s)
 {
+    const double alpha = (double)alpha_f;
     if (!amax || !wmax || !s || K <= 0 || !(alpha >= 0.0 && alpha <= 1.0)) return ZQO_EARG;
     for (int64_t j = 0; j < K; ++j) {
         if (amax[j] == 0.0f || wmax[j] == 0.0f) {

@@ -213,6 +213,37 @@ int zq_quantize_weights(const float* W, int64_t N, int64_t K, int64_t group_rows
     return launch_quantize_weights(W, N, K, group_rows, Wq, s_grp, di, as_stream(stream));
 }
 
+int zq_smooth_calibrate(const void* x, int x_dtype, int64_t T, int64_t H, const float* gamma,
+                        const float* beta, float eps, float* amax, void* stream) {
+    if (!x || !amax) return ZQ_ERR_NULL;
+    if (x_dtype != ZQ_F32 && x_dtype != ZQ_BF16) return ZQ_ERR_DTYPE;
+    // H <= 32768: the kernel keeps one maximum per channel in shared memory
+    if (T <= 0 || H <= 0 || H % 16 != 0 || H > 32768 || T > ((int64_t)1 << 31) - 32) return ZQ_ERR_SHAPE;
+    if (!aligned(x, 16) || !aligned(amax, 4) || (gamma && !aligned(gamma, 4)) || (beta && !aligned(beta, 4)))
+        return ZQ_ERR_ALIGN;
+    DeviceInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    return launch_smooth_calibrate(x, x_dtype, T, H, gamma, gamma ? beta : nullptr, eps, amax, di, as_stream(stream));
+}
+
+int zq_smooth_weights(const float* W, int64_t N, int64_t K, const float* amax, float alpha, const float* gamma,
+                      const float* beta, float* W_out, float* gamma_out, float* beta_out, float* s, void* stream) {
+    if (!W || !amax || !W_out || !s) return ZQ_ERR_NULL;
+    if ((gamma && !gamma_out) || (beta && !beta_out)) return ZQ_ERR_NULL;
+    if (!(alpha >= 0.0f && alpha <= 1.0f)) return ZQ_ERR_DTYPE;
+    if (N <= 0 || K <= 0 || K % 16 != 0 || N > ((int64_t)1 << 40) / K) return ZQ_ERR_SHAPE;
+    if (!aligned(W, 16) || !aligned(W_out, 16) || !aligned(s, 16) || !aligned(amax, 4)) return ZQ_ERR_ALIGN;
+    if ((gamma && !aligned(gamma, 4)) || (beta && !aligned(beta, 4)) || (gamma_out && !aligned(gamma_out, 4)) ||
+        (beta_out && !aligned(beta_out, 4)))
+        return ZQ_ERR_ALIGN;
+    DeviceInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    return launch_smooth_weights(W, N, K, amax, alpha, gamma, beta, W_out, gamma_out, beta_out, s, di,
+                                 as_stream(stream));
+}
+
 int zq_ln_quant(const void* x, int x_dtype, int64_t T, int64_t H, const float* gamma,
                 const float* beta, float eps, int8_t* q, float* s_tok, void* stream) {
     int rc = check_rows(x, x_dtype, T, H, q, s_tok);

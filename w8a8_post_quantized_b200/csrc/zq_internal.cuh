@@ -627,6 +627,11 @@ int launch_rowq_pipe(const void* x, int x_dtype, int64_t T, int64_t H, bool ln, 
                      float* s_tok, const DeviceInfo& di, cudaStream_t st);
 int launch_requant_rows(const float* h, int64_t T, int64_t N, const uint32_t* amax_bits, int8_t* q,
                         float* s_tok, const DeviceInfo& di, cudaStream_t st);
+int launch_smooth_calibrate(const void* x, int x_dtype, int64_t T, int64_t H, const float* gamma,
+                            const float* beta, float eps, float* amax, const DeviceInfo& di, cudaStream_t st);
+int launch_smooth_weights(const float* W, int64_t N, int64_t K, const float* amax, float alpha, const float* gamma,
+                          const float* beta, float* W_out, float* gamma_out, float* beta_out, float* s,
+                          const DeviceInfo& di, cudaStream_t st);
 
 struct LinearArgs {
     const int8_t* xq;

@@ -33,7 +33,7 @@ EXPORTED = (
     "zq_quantize_weights", "zq_ln_quant", "zq_act_quant", "zq_w8a8_linear_workspace",
     "zq_w8a8_linear", "zq_linear_block_workspace", "zq_linear_block", "zq_device_status",
     "zq_status_string", "zq_last_cuda_error", "zq_version", "zq_launch_count",
-    "zq_w8a8_linear_requant_noalloc",
+    "zq_w8a8_linear_requant_noalloc", "zq_smooth_calibrate", "zq_smooth_weights",
 )
 
 
@@ -73,6 +73,8 @@ def lib() -> ctypes.CDLL:
         "zq_version": (I, []),
         "zq_launch_count": (ctypes.c_uint64, []),
         "zq_w8a8_linear_requant_noalloc": (I, [P, P, I64, I64, P, P, I64, I64, P, I, P, P, P]),
+        "zq_smooth_calibrate": (I, [P, I, I64, I64, P, P, F, P, P]),
+        "zq_smooth_weights": (I, [P, I64, I64, P, F, P, P, P, P, P, P, P]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -129,6 +131,32 @@ def zq_ln_quant(x, gamma, beta, eps, q=None, s_tok=None, stream=None):
     _check(lib().zq_ln_quant(_p(x), _dtype_code(x), T, H, _p(gamma), _p(beta), float(eps),
                              _p(q), _p(s_tok), _s(stream)), "zq_ln_quant")
     return q, s_tok
+
+
+def zq_smooth_calibrate(x, gamma=None, beta=None, eps=1e-5, amax=None, stream=None):
+    """Running per-channel absmax of LayerNorm(x) (or x without gamma); pass
+    the returned amax back in for the next calibration batch."""
+    T, H = x.shape
+    amax = torch.zeros(H, dtype=torch.float32, device=x.device) if amax is None else amax
+    _check(lib().zq_smooth_calibrate(_p(x), _dtype_code(x), T, H, _p(gamma), _p(beta), float(eps),
+                                     _p(amax), _s(stream)), "zq_smooth_calibrate")
+    return amax
+
+
+def zq_smooth_weights(W, amax, alpha=0.5, gamma=None, beta=None, W_out=None, gamma_out=None,
+                      beta_out=None, s=None, stream=None):
+    """SmoothQuant factors and fold: returns (W_out, gamma_out, beta_out, s)."""
+    N, K = W.shape
+    W_out = torch.empty_like(W) if W_out is None else W_out
+    if gamma is not None and gamma_out is None:
+        gamma_out = torch.empty_like(gamma)
+    if beta is not None and beta_out is None:
+        beta_out = torch.empty_like(beta)
+    s = torch.empty(K, dtype=torch.float32, device=W.device) if s is None else s
+    _check(lib().zq_smooth_weights(_p(W), N, K, _p(amax), float(alpha), _p(gamma), _p(beta),
+                                   _p(W_out), _p(gamma_out), _p(beta_out), _p(s), _s(stream)),
+           "zq_smooth_weights")
+    return W_out, gamma_out, beta_out, s
 
 
 def zq_act_quant(x, bias=None, act=ZQ_ACT_NONE, q=None, s_tok=None, stream=None):
