@@ -127,14 +127,25 @@ struct Team {
     }
     // Merge per-thread (count, mean, sum of squared deviations) over the team
     // with Chan's pairwise update; returns the team's mean and M2.
+    // EQ: every thread holds the same count n, so each merge joins two equal
+    // halves: mean = (mean_a + mean_b) / 2, M2 = M2_a + M2_b + d^2 n / 2
+    // (Chan's update with n_a = n_b; no division).
+    template <bool EQ = false>
     static __device__ __forceinline__ void stats(float n, float mean, float m2, float* red, int team,
                                                  float& mean_out, float& m2_out) {
 #pragma unroll
         for (int o = kTopLane; o > 0; o >>= 1) {
-            const float nb = __shfl_xor_sync(0xFFFFFFFFu, n, o);
             const float mb = __shfl_xor_sync(0xFFFFFFFFu, mean, o);
             const float qb = __shfl_xor_sync(0xFFFFFFFFu, m2, o);
-            merge(n, mean, m2, nb, mb, qb);
+            if constexpr (EQ) {
+                const float d = mb - mean;
+                mean = fmaf(0.5f, d, mean);
+                m2 = m2 + qb + d * d * (0.5f * n);
+                n = n + n;
+            } else {
+                const float nb = __shfl_xor_sync(0xFFFFFFFFu, n, o);
+                merge(n, mean, m2, nb, mb, qb);
+            }
         }
         if constexpr (TPR > 32) {
             constexpr int W = TPR / 32;
@@ -186,7 +197,11 @@ struct Team {
     }
 };
 
-template <typename Tin, bool LN, int TPR, int PPT, int BLOCK, bool SMEMP>
+// FULL: the row is exactly TPR * PPT pieces, so every piece of every row a
+// team touches exists; the per-piece guards vanish at compile time (rows past
+// the block's end are computed on row 0's data and only their stores are
+// skipped).
+template <typename Tin, bool LN, int TPR, int PPT, int BLOCK, bool SMEMP, bool FULL>
 __global__ void __launch_bounds__(BLOCK, 1)
 rowq_pipe_kernel(const Tin* __restrict__ x, int T, int H, float inv_h, int R, int nstages,
                  const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
@@ -205,7 +220,7 @@ rowq_pipe_kernel(const Tin* __restrict__ x, int T, int H, float inv_h, int R, in
     uint8_t* ring = smem + kRingOffset + (SMEMP ? (size_t)n_par * H * sizeof(float) : 0);
     const int row_bytes = H * (int)sizeof(Tin);
     const int stage_bytes = R * row_bytes;
-    const int nP = H / EPP;
+    const int nP = FULL ? TPR * PPT : H / EPP;  // pieces per row (compile-time when exact)
     const int team = threadIdx.x / TPR;
     const int tt = threadIdx.x % TPR;
     const int n_units = (T + R - 1) / R;
@@ -279,7 +294,7 @@ rowq_pipe_kernel(const Tin* __restrict__ x, int T, int H, float inv_h, int R, in
 #pragma unroll
             for (int k = 0; k < PPT; ++k) {
                 const int p = k * TPR + tt;
-                okp[k] = row_ok && p < nP;
+                okp[k] = FULL || (row_ok && p < nP);
                 if (okp[k]) Piece<Tin>::load(xr + p * EPP, v[k]);
                 else {
 #pragma unroll
@@ -314,8 +329,9 @@ rowq_pipe_kernel(const Tin* __restrict__ x, int T, int H, float inv_h, int R, in
                         }
                     }
                 float mean, m2;
-                TM::stats(n_loc, mean_loc, f2_hsum(f2_add(f2_add(da[0], da[1]), f2_add(da[2], da[3]))),
-                          red, team, mean, m2);
+                TM::template stats<FULL>(n_loc, mean_loc,
+                                         f2_hsum(f2_add(f2_add(da[0], da[1]), f2_add(da[2], da[3]))), red, team,
+                                         mean, m2);
                 const float rstd = rsqrtf(fmaf(m2, inv_h, eps));
                 const uint64_t mean2 = f2_pack(mean, mean);
                 const uint64_t rstd2 = f2_pack(rstd, rstd);
@@ -368,11 +384,11 @@ rowq_pipe_kernel(const Tin* __restrict__ x, int T, int H, float inv_h, int R, in
             if (LN || act == ZQ_ACT_GELU) {
 #pragma unroll
                 for (int k = 0; k < PPT; ++k)
-                    if (okp[k]) store_piece_codes<NP, true>(qr + (k * TPR + tt) * EPP, v[k], inv2);
+                    if (FULL ? row_ok : okp[k]) store_piece_codes<NP, true>(qr + (k * TPR + tt) * EPP, v[k], inv2);
             } else {
 #pragma unroll
                 for (int k = 0; k < PPT; ++k)
-                    if (okp[k]) store_piece_codes<NP, false>(qr + (k * TPR + tt) * EPP, v[k], inv2);
+                    if (FULL ? row_ok : okp[k]) store_piece_codes<NP, false>(qr + (k * TPR + tt) * EPP, v[k], inv2);
             }
             if (row_ok && tt == 0) s_tok[row] = scale;
         }
@@ -402,22 +418,28 @@ constexpr Shape kShapes[] = {{16, 1, 512},   {16, 2, 512},  {16, 4, 512},  {16, 
 constexpr int kNumShapes = 12;
 constexpr int kFirstGlobalParamShape = 10;  // from here on parameters stay in global memory
 
-template <typename Tin, bool LN>
-PipeKernel<Tin, LN> pipe_kernel(int idx) {
+template <typename Tin, bool LN, bool FULL>
+PipeKernel<Tin, LN> pipe_kernel_t(int idx) {
     switch (idx) {
-        case 0: return rowq_pipe_kernel<Tin, LN, 16, 1, 512, true>;
-        case 1: return rowq_pipe_kernel<Tin, LN, 16, 2, 512, true>;
-        case 2: return rowq_pipe_kernel<Tin, LN, 16, 4, 512, true>;
-        case 3: return rowq_pipe_kernel<Tin, LN, 16, 6, 512, true>;
-        case 4: return rowq_pipe_kernel<Tin, LN, 16, 8, 512, true>;
-        case 5: return rowq_pipe_kernel<Tin, LN, 32, 8, 512, true>;
-        case 6: return rowq_pipe_kernel<Tin, LN, 64, 8, 512, true>;
-        case 7: return rowq_pipe_kernel<Tin, LN, 128, 6, 512, true>;
-        case 8: return rowq_pipe_kernel<Tin, LN, 128, 8, 512, true>;
-        case 9: return rowq_pipe_kernel<Tin, LN, 256, 6, 512, true>;
-        case 10: return rowq_pipe_kernel<Tin, LN, 256, 8, 512, false>;
-        default: return rowq_pipe_kernel<Tin, LN, 256, 16, 256, false>;
+        case 0: return rowq_pipe_kernel<Tin, LN, 16, 1, 512, true, FULL>;
+        case 1: return rowq_pipe_kernel<Tin, LN, 16, 2, 512, true, FULL>;
+        case 2: return rowq_pipe_kernel<Tin, LN, 16, 4, 512, true, FULL>;
+        case 3: return rowq_pipe_kernel<Tin, LN, 16, 6, 512, true, FULL>;
+        case 4: return rowq_pipe_kernel<Tin, LN, 16, 8, 512, true, FULL>;
+        case 5: return rowq_pipe_kernel<Tin, LN, 32, 8, 512, true, FULL>;
+        case 6: return rowq_pipe_kernel<Tin, LN, 64, 8, 512, true, FULL>;
+        case 7: return rowq_pipe_kernel<Tin, LN, 128, 6, 512, true, FULL>;
+        case 8: return rowq_pipe_kernel<Tin, LN, 128, 8, 512, true, FULL>;
+        case 9: return rowq_pipe_kernel<Tin, LN, 256, 6, 512, true, FULL>;
+        case 10: return rowq_pipe_kernel<Tin, LN, 256, 8, 512, false, false>;
+        default: return rowq_pipe_kernel<Tin, LN, 256, 16, 256, false, false>;
     }
+}
+
+// The kernel for shape idx; full: the row is exactly the shape's TPR * PPT pieces.
+template <typename Tin, bool LN>
+PipeKernel<Tin, LN> pipe_kernel(int idx, bool full) {
+    return full ? pipe_kernel_t<Tin, LN, true>(idx) : pipe_kernel_t<Tin, LN, false>(idx);
 }
 
 // Smallest shape whose team covers the row's pieces.
@@ -453,7 +475,10 @@ int launch_typed(const Tin* x, int64_t T, int64_t H, const float* gamma, const f
     const int64_t n_units = (T + R - 1) / R;
     const int grid = (int)(n_units < di.sm_count ? n_units : di.sm_count);
     const size_t smem = kRingOffset + par_bytes + (size_t)nstages * stage_bytes;
-    auto kern = pipe_kernel<Tin, LN>(idx);
+    // exact-fit rows drop the per-piece guards (not for the global-parameter
+    // shapes, whose guard-free variants need more registers than they have)
+    const bool full = (int64_t)sh.tpr * sh.ppt * EPP == H && idx < kFirstGlobalParamShape;
+    auto kern = pipe_kernel<Tin, LN>(idx, full);
     int rc = cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     if (rc) return rc;
     cudaLaunchConfig_t cfg = {};
