@@ -197,7 +197,7 @@ def weight_col_absmax(W):
 
 
 def smooth_factors(amax, wmax, alpha=0.5):
-    """s_j = amax_j^alpha / wmax_j^(1-alpha) (reading R9 of zq_oracle.c);
+    """s_j = amax_j^alpha / wmax_j^(1-alpha) (reading R14 of zq_oracle.c);
     alpha is taken as an fp32 value, as the library's interface passes it."""
     a, pa = _c(amax, np.float32)
     w, pw = _c(wmax, np.float32)

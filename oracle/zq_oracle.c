@@ -45,13 +45,13 @@
  *   R6 LayerNorm uses the biased variance with eps inside the square root;
  *   R7 GeLU is the exact erf form 0.5 x (1 + erf(x / sqrt 2));
  *   R8 bias is added after dequantization, in floating point.
- *   R9 the smoothing factor is the SmoothQuant paper's balance rule (the
+ *  R14 the smoothing factor is the SmoothQuant paper's balance rule (the
  *      pages name the paper but are cut off before its formula):
  *      s_j = amax_x[j]^alpha / amax_w[j]^(1 - alpha), alpha the migration
  *      strength (0.5 balances both maxima; 1 equalises the activation
  *      channels); computed in double, rounded to fp32, at least 1e-5; a
  *      channel whose activation or weight absmax is 0 keeps s_j = 1;
- *  R10 the activation diag(s)^-1 is folded into the preceding LayerNorm's
+ *  R15 the activation diag(s)^-1 is folded into the preceding LayerNorm's
  *      gamma and beta (the normalised row is divided per channel), so the
  *      online path is unchanged.
  *
@@ -232,7 +232,7 @@ int zqo_weight_col_absmax(const float* W, int64_t N, int64_t K, float* wmax)
     return ZQO_OK;
 }
 
-/* [TS36] §1.3 / [SQ] §2.2, reading R9: s_j = amax_j^alpha / wmax_j^(1-alpha).
+/* [TS36] §1.3 / [SQ] §2.2, reading R14: s_j = amax_j^alpha / wmax_j^(1-alpha).
  * alpha is an fp32 parameter (the migration strength as the library's
  * interface passes it); the powers use its exact value in double. */
 int zqo_smooth_factors(const float* amax, const float* wmax, int64_t K, float alpha_f, float* s)
@@ -251,7 +251,7 @@ int zqo_smooth_factors(const float* amax, const float* wmax, int64_t K, float al
     return ZQO_OK;
 }
 
-/* [TS36] §1.3 identity, reading R10: W_out[o, j] = W[o, j] * s_j (each
+/* [TS36] §1.3 identity, reading R15: W_out[o, j] = W[o, j] * s_j (each
  * output row scaled per input channel), gamma_out[j] = gamma[j] / s_j,
  * beta_out[j] = beta[j] / s_j; each computed in double and rounded once to
  * fp32 (gamma or beta may be NULL: not folded). */

@@ -4,7 +4,7 @@ Sources: "探秘Transformer系列之（36）— 大模型量化方案" §1.3 and
 "SmoothQuant技术解析：大模型INT8量化的突破与实践" §2.2, §3: the output is
 unchanged by Y = (X diag(s)^-1)(diag(s) W); s is chosen per channel offline
 so that the smoothed activation channels have similar maxima; the maxima come
-from calibration batches.  The factor rule (reading R9 of the oracle) is the
+from calibration batches.  The factor rule (reading R14 of the oracle) is the
 SmoothQuant paper's s_j = amax_j^alpha / wmax_j^(1-alpha).
 
 Pins: hand-worked factors (``tests/golden/smooth_factors.txt``); the balance

@@ -377,8 +377,8 @@ rowq_pipe_kernel(const Tin* __restrict__ x, int T, int H, float inv_h, int R, in
                 amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
             }
             amax = TM::max(amax, red, team);
-            float scale, inv;
-            absmax_scales(amax, scale, inv);
+            // inv = 127/amax for every thread; scale = amax/127 only where it is stored
+            const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
             const uint64_t inv2 = f2_pack(inv, inv);
             int8_t* qr = q + row * H;
             if (LN || act == ZQ_ACT_GELU) {
@@ -390,7 +390,7 @@ rowq_pipe_kernel(const Tin* __restrict__ x, int T, int H, float inv_h, int R, in
                 for (int k = 0; k < PPT; ++k)
                     if (FULL ? row_ok : okp[k]) store_piece_codes<NP, false>(qr + (k * TPR + tt) * EPP, v[k], inv2);
             }
-            if (row_ok && tt == 0) s_tok[row] = scale;
+            if (row_ok && tt == 0) s_tok[row] = __fdiv_rn(amax, 127.0f);
         }
         __syncthreads();  // every team is done with stage s
         if (threadIdx.x == 0) {
