@@ -184,7 +184,13 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     if (SWAP) cluster_sync_all();  // peers' barriers initialised before any remote arrive
-    griddep_wait();                // inputs and outputs are free of the previous grid in the stream
+    // Programmatic dependent launch.  The weights (codes, group scales, bias)
+    // are never written by a kernel that lets its successor start early (the
+    // hot-path kernels that trigger early write only activations and outputs;
+    // the weight preparation kernels run to completion first), so the
+    // producer streams the first ring of weight tiles before waiting for the
+    // previous grid; every role waits before it touches activations or
+    // outputs.
     griddep_launch_dependents();
     const uint32_t tmem_base = *tmem_slot;
 
@@ -199,6 +205,27 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
+            // the weight operand is A when the roles are swapped, else B
+            auto load_w = [&](int s, int kb, int mt, int nt) {
+                if (SWAP) tma_load_2d(sA + s * A_STAGE, &tmA, bar_full(s), kb * BK, mt * BM);
+                else tma_load_2d(sB + s * B_STAGE, &tmB, bar_full(s), kb * BK, nt * BN);
+            };
+            auto load_x = [&](int s, int kb, int mt, int nt) {
+                if (SWAP) tma_load_2d(sB + s * B_STAGE, &tmB, bar_full(s), kb * BK, nt * BN);
+                else tma_load_2d(sA + s * A_STAGE, &tmA, bar_full(s), kb * BK, mt * BM);
+            };
+            // first ring fill: the weight halves of the first STAGES stages
+            // (their slots are free), before the wait for the previous grid
+            uint32_t npre = 0;
+            for (int tile = cl; npre < (uint32_t)STAGES && tile < num_tiles; tile += ncl) {
+                int mt, nt;
+                tile_coords(tile, m_tiles, n_tiles, p.group_m, mt, nt);
+                for (int kb = kb_begin; kb < kb_end && npre < (uint32_t)STAGES; ++kb, ++npre) {
+                    mbar_arrive_expect_tx(bar_full((int)npre), A_STAGE + B_STAGE);
+                    load_w((int)npre, kb, mt, nt);
+                }
+            }
+            griddep_wait();
             uint32_t it = 0;
             bool ok = true;
             for (int tile = cl; ok && tile < num_tiles; tile += ncl) {
@@ -207,13 +234,15 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1u;
-                    if (!mbar_wait(bar_empty(s), ph ^ 1u, abort_flag, p.status, SITE_PRODUCER_EMPTY)) {
-                        ok = false;
-                        break;
+                    if (it >= npre) {
+                        if (!mbar_wait(bar_empty(s), ph ^ 1u, abort_flag, p.status, SITE_PRODUCER_EMPTY)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(bar_full(s), A_STAGE + B_STAGE);
+                        load_w(s, kb, mt, nt);
                     }
-                    mbar_arrive_expect_tx(bar_full(s), A_STAGE + B_STAGE);
-                    tma_load_2d(sA + s * A_STAGE, &tmA, bar_full(s), kb * BK, mt * BM);
-                    tma_load_2d(sB + s * B_STAGE, &tmB, bar_full(s), kb * BK, nt * BN);
+                    load_x(s, kb, mt, nt);
                 }
             }
             // Let every copy this thread issued land before the CTA can exit:
@@ -264,6 +293,7 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         __syncwarp();
     } else {
         // ------------------------------------------------ epilogue
+        griddep_wait();  // token scales are the previous grid's output; y may still be read by it
         // warp w may only read TMEM lanes 32*(w%4) .. +31; EW/4 warps share each
         // lane quarter and split the tile's columns between them
         constexpr int SLICES = EW / 4;

@@ -192,8 +192,7 @@ weight_col_absmax_kernel(const float* __restrict__ W, int64_t N, int64_t K, uint
 __global__ void __launch_bounds__(256)
 smooth_factor_kernel(const float* __restrict__ amax, float* s, int64_t K, double alpha, const float* gamma,
                      const float* beta, float* gamma_out, float* beta_out) {
-    griddep_wait();
-    griddep_launch_dependents();
+    griddep_wait();  // writes weights / parameters: successors start only at completion
     const int64_t j = (int64_t)blockIdx.x * 256 + threadIdx.x;
     if (j >= K) return;
     const float a = amax[j], w = s[j];
@@ -211,8 +210,7 @@ smooth_factor_kernel(const float* __restrict__ amax, float* s, int64_t K, double
 // W_out[o, j] = W[o, j] * s[j] (one fp32 rounding of the exact product).
 __global__ void __launch_bounds__(256)
 smooth_fold_kernel(const float* W, int64_t N, int64_t K, const float* __restrict__ s, float* W_out) {
-    griddep_wait();
-    griddep_launch_dependents();
+    griddep_wait();  // writes weights / parameters: successors start only at completion
     const int64_t n4 = N * K / 4;  // K % 16 == 0: rows are whole float4s
     const int64_t k4 = K / 4;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
