@@ -35,6 +35,8 @@ GEMM_SHAPES = [
     (16, 64, 256, 16),       # the tiny layer: swapped, BN = 16, K < one stage
     (1, 160, 128, 128),      # one token, K = 128 + 32
     (33, 4096, 384, 128),    # swapped, BN = 64 (33 tokens)
+    (24, 6144, 1024, 128),   # swapped, BN = 32 (16-column epilogue chunks), split K
+    (32, 2048, 272, 16),     # swapped, BN = 32, ragged M tile
     (64, 1040, 272, 16),     # swapped, N % 32 == 16, K tail of 16
     (65, 256, 512, 64),      # first non-swapped T
     (200, 384, 512, 64),     # ragged T

@@ -114,7 +114,9 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     static_assert(EW % 4 == 0 && EW >= 4 && EW <= 16, "epilogue warps cover the 4 TMEM lane quarters");
     constexpr int kEpiThreads = 32 * EW;
     constexpr int B_STAGE = BN * BK;
-    constexpr int CW = (BN % 32 == 0) ? 32 : 16;  // epilogue column chunk
+    // epilogue column chunk (16 for the swapped 32-token tile: 32 there spills
+    // registers next to the split-K partial sums)
+    constexpr int CW = (BN % 32 == 0 && !(SWAP && BN == 32)) ? 32 : 16;
     constexpr uint32_t IDESC = idesc_i8(BM, BN);
     constexpr uint32_t TMEM_COLS = tmem_cols<BN>();
 
