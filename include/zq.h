@@ -49,6 +49,18 @@
  *     kernel records the fact in a device flag and returns early (output
  *     undefined); zq_device_status() reports it as ZQ_ERR_TIMEOUT.
  *   - NaN or Inf inputs are outside the contract (not checked on device).
+ *   - Hot-path kernels are launched with programmatic dependent launch:
+ *     a kernel may start while the previous kernel on the stream finishes
+ *     and waits (griddepcontrol.wait) before it reads activations or writes
+ *     outputs.  The W8A8 linear starts streaming its weights (Wq, s_grp,
+ *     bias) before that wait, so the weights must not be written by a kernel
+ *     that lets its successors start early (none of this library's kernels
+ *     does; zq_quantize_weights and zq_smooth_weights finish first).  Set
+ *     ZQ_NO_PDL in the environment to launch every kernel in plain stream
+ *     order.
+ *   - The SmoothQuant entry points (zq_smooth_calibrate, zq_smooth_weights)
+ *     cover [TS36] §1.3 and "SmoothQuant技术解析：大模型INT8量化的突破与实践";
+ *     see their declarations.
  */
 #ifndef ZQ_H_
 #define ZQ_H_
