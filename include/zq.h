@@ -263,8 +263,18 @@ int zq_smooth_weights(const float* W, int64_t N, int64_t K, const float* amax, f
  * calls (static storage, "no error" when none).
  * zq_version: library version as 10000*major + 100*minor + patch.
  * zq_launch_count: number of kernels this library has launched in this
- * process (all devices, all threads); for accounting in benchmarks. */
+ * process (all devices, all threads); for accounting in benchmarks.
+ * zq_watchdog_selftest: see below. */
 int zq_device_status(void* stream);
+/* zq_watchdog_selftest: enqueues one tiny kernel whose only thread waits on
+ * a barrier that nothing signals.  Its bounded wait expires after the
+ * library's wait limit (about 2 s), records a site code in the device flag
+ * and returns, exactly as an expired wait inside the GEMM does; the next
+ * zq_device_status() then reports ZQ_ERR_TIMEOUT (and clears the flag) and
+ * the CUDA context stays usable.  It exists to test that failure path
+ * without faulting or hanging the GPU.  Returns ZQ_OK, ZQ_ERR_CUDA or
+ * ZQ_ERR_DEVICE. */
+int zq_watchdog_selftest(void* stream);
 const char* zq_status_string(int status);
 const char* zq_last_cuda_error(void);
 int zq_version(void);

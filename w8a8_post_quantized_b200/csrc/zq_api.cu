@@ -185,6 +185,33 @@ const char* zq_status_string(int status) {
 
 const char* zq_last_cuda_error(void) { return t_last_error; }
 
+namespace zq {
+namespace {
+constexpr int kSiteWatchdogSelftest = 0x7E57;
+// One thread waits on an mbarrier that nothing arrives on: the bounded wait
+// expires after its limit, records the site in the status word and returns.
+__global__ void watchdog_selftest_kernel(int* status) {
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t b = smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        mbar_init(b, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(b, 0u, nullptr, status, kSiteWatchdogSelftest);
+}
+}  // namespace
+}  // namespace zq
+
+int zq_watchdog_selftest(void* stream) {
+    DeviceInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    count_launch();
+    watchdog_selftest_kernel<<<1, 32, 0, as_stream(stream)>>>(di.status_word);
+    return cuda_status(cudaGetLastError());
+}
+
 int zq_device_status(void* stream) {
     DeviceInfo di;
     int rc = device_info(&di);

@@ -34,6 +34,7 @@ EXPORTED = (
     "zq_w8a8_linear", "zq_linear_block_workspace", "zq_linear_block", "zq_device_status",
     "zq_status_string", "zq_last_cuda_error", "zq_version", "zq_launch_count",
     "zq_w8a8_linear_requant_noalloc", "zq_smooth_calibrate", "zq_smooth_weights",
+    "zq_watchdog_selftest",
 )
 
 
@@ -75,6 +76,7 @@ def lib() -> ctypes.CDLL:
         "zq_w8a8_linear_requant_noalloc": (I, [P, P, I64, I64, P, P, I64, I64, P, I, P, P, P]),
         "zq_smooth_calibrate": (I, [P, I, I64, I64, P, P, F, P, P]),
         "zq_smooth_weights": (I, [P, I64, I64, P, F, P, P, P, P, P, P, P]),
+        "zq_watchdog_selftest": (I, [P]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -232,6 +234,12 @@ def zq_w8a8_linear_requant_noalloc(xq, s_tok, Wq, s_grp, group_rows, bias=None,
 
 def zq_device_status(stream=None):
     _check(lib().zq_device_status(_s(stream)), "zq_device_status")
+
+
+def zq_watchdog_selftest(stream=None):
+    """Enqueue a kernel whose bounded wait expires (about 2 s); the next
+    zq_device_status() raises ZQError with ZQ_ERR_TIMEOUT."""
+    _check(lib().zq_watchdog_selftest(_s(stream)), "zq_watchdog_selftest")
 
 
 def zq_version() -> int:
