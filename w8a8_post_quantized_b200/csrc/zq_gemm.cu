@@ -452,9 +452,14 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(bar_tempty(b));
-                        fence_acq_rel_cluster();
+                        // every thread's partials are ordered before this CTA barrier;
+                        // one cluster-scope fence by the arriving thread then
+                        // releases them all to the leader (cumulativity)
                         named_bar_sync(1, kEpiThreads);
-                        if (et == 0) mbar_arrive_cluster(mapa_shared(bar_red_full(b), 0u));
+                        if (et == 0) {
+                            fence_acq_rel_cluster();
+                            mbar_arrive_cluster(mapa_shared(bar_red_full(b), 0u));
+                        }
                         continue;
                     }
                 }
