@@ -16,6 +16,7 @@ Sources (web pages):
          fake quantization, quantization error.
   [SQ]   "SmoothQuant技术解析：大模型INT8量化的突破与实践" §2.2, §3 and [TS36]
          §1.3 -- per-channel smoothing folded offline into the weights.
+  [TS36] §1.1 LLM.int8() -- mixed-precision decomposition of outlier columns.
 
 Every function here is pinned by ``tests/test_oracle_pins.py`` against
 hand-worked examples (``tests/golden/``), closed forms, invariants and
@@ -70,11 +71,15 @@ def _L():
             "zqo_weight_col_absmax": [P, I64, I64, P],
             "zqo_smooth_factors": [P, P, I64, F, P],
             "zqo_smooth_fold": [P, I64, I64, P, P, P, P, P, P],
+            "zqo_outlier_product": [P, I64, I64, P, I64, P, I64, P],
+            "zqo_dequant_add": [P, I64, I64, P, P, I64, P, P, ctypes.c_int, P],
         }
         for name, args in sig.items():
             fn = getattr(lib, name)
             fn.argtypes = args
             fn.restype = ctypes.c_int
+        lib.zqo_outlier_columns.argtypes = [P, I64, F, P, I64]
+        lib.zqo_outlier_columns.restype = I64
         _lib = lib
     return _lib
 
@@ -269,3 +274,64 @@ def smooth_ln_linear(calib_batches, gamma, beta, eps, W, alpha=0.5):
     s = smooth_factors(amax, weight_col_absmax(W), alpha)
     Wo, go, bo = smooth_fold(W, s, gamma, beta)
     return Wo, go, bo, s, amax
+
+
+# ---- LLM.int8() mixed-precision decomposition ([TS36] §1.1, reading R16) ---
+
+LLM_INT8_ALPHA = 6.0
+
+
+def outlier_columns(amax, threshold=LLM_INT8_ALPHA, max_o=8):
+    """Columns with amax >= threshold, ascending; returns (first max_o of them, total count)."""
+    a, pa = _c(amax, np.float32)
+    idx = np.zeros(max(max_o, 1), np.int32)
+    n = _L().zqo_outlier_columns(pa, a.size, float(threshold), idx.ctypes.data, int(max_o))
+    if n < 0:
+        raise OracleError("outlier_columns: bad argument")
+    return idx[:min(n, max_o)].copy(), int(n)
+
+
+def outlier_product(a, W, idx):
+    """sum over the listed columns j of fp16(a[t, j]) * fp16(W[o, j]), in float64."""
+    a, pa = _c(a, np.float32)
+    W, pw = _c(W, np.float32)
+    ix, pi = _c(idx, np.int32)
+    T, K = a.shape
+    N = W.shape[0]
+    out = np.empty((T, N), np.float64)
+    _chk(_L().zqo_outlier_product(pa, T, K, pw, N, pi if ix.size else None, ix.size, out.ctypes.data),
+         "outlier_product")
+    return out
+
+
+def dequant_add(acc, s_tok, s_grp, group_rows, add=None, bias=None, act=ACT_NONE):
+    """y = act(s_tok s_grp acc + add + bias) in double -> fp32."""
+    acc, pa = _c(acc, np.int32)
+    st, ps = _c(s_tok, np.float32)
+    sg, pg = _c(s_grp, np.float32)
+    T, N = acc.shape
+    pad = pb = None
+    if add is not None:
+        add, pad = _c(add, np.float64)
+    if bias is not None:
+        bias, pb = _c(bias, np.float32)
+    y = np.empty((T, N), np.float32)
+    _chk(_L().zqo_dequant_add(pa, T, N, ps, pg, group_rows, pad, pb, int(act), y.ctypes.data), "dequant_add")
+    return y
+
+
+def int8_decomposed_ln_linear(x, gamma, beta, eps, W, Wq, s_grp, group_rows, bias=None, act=ACT_NONE,
+                              threshold=LLM_INT8_ALPHA, max_o=8):
+    """LLM.int8() on a LayerNorm-fed linear: detect the outlier columns of the
+    LayerNorm output over the batch, quantize the other columns per token
+    (the outlier columns contribute zero codes), run the INT8 GEMM with the
+    group-quantized weights, add the fp16 outlier product, then bias and
+    activation.  Returns (y fp32, outlier columns, total outlier count)."""
+    a = layernorm(x, gamma, beta, eps)
+    idx, n = outlier_columns(channel_absmax(a), threshold, max_o)
+    a_in = a.copy()
+    a_in[:, idx] = 0.0
+    xq, st = quantize_rows(a_in)
+    add = outlier_product(a, W, idx)
+    y = dequant_add(gemm_i32(xq, Wq), st, s_grp, group_rows, add, bias, act)
+    return y, idx, n

@@ -30,6 +30,12 @@
  *   [TS36] §1.3 SmoothQuant -- per-channel smoothing factor s chosen
  *          offline; Y = (X diag(s)^-1)(diag(s) W): weights scaled up per
  *          input channel, activations scaled down, output unchanged.
+ *   [TS36] §1.1 LLM.int8() -- mixed-precision decomposition: the columns
+ *          of the input holding a value above the threshold alpha = 6.0
+ *          form the outlier set O; X[:, O] times the matching weights run in
+ *          FP16; the other columns are quantized (absmax per row of X and
+ *          per output of W) for the INT8 product, dequantized, and the two
+ *          results are added.
  *   [SQ]   "SmoothQuant技术解析：大模型INT8量化的突破与实践" §2.2 (the same
  *          identity; s chosen so the channels of X diag(s)^-1 have similar
  *          absolute maxima), §3 (calibration of per-channel max |X| over
@@ -54,6 +60,14 @@
  *  R15 the activation diag(s)^-1 is folded into the preceding LayerNorm's
  *      gamma and beta (the normalised row is divided per channel), so the
  *      online path is unchanged.
+ *  R16 LLM.int8() outliers are detected on the linear's input (after the
+ *      LayerNorm) over the whole batch: column j is in O when some
+ *      |a[t, j]| >= alpha; at most max_o columns (the lowest indices) are
+ *      decomposed; the weights keep their offline group quantization over
+ *      all input channels (the outlier channels see zero activation codes);
+ *      the outlier operands are rounded to fp16 (round to nearest even) and
+ *      multiplied exactly; the outlier product is added to the dequantized
+ *      INT8 result before bias and activation.
  *
  * Status codes: 0 = ok, 1 = bad argument, 2 = int32 overflow in the GEMM.
  */
@@ -266,5 +280,78 @@ int zqo_smooth_fold(const float* W, int64_t N, int64_t K, const float* gamma, co
         if (gamma) gamma_out[j] = (float)((double)gamma[j] / (double)s[j]);
         if (beta) beta_out[j] = (float)((double)beta[j] / (double)s[j]);
     }
+    return ZQO_OK;
+}
+
+/* [TS36] §1.1 outlier detection, reading R16: the columns j with
+ * amax[j] >= threshold in ascending order, at most max_o of them written;
+ * returns the total count. */
+int64_t zqo_outlier_columns(const float* amax, int64_t K, float threshold, int32_t* idx, int64_t max_o)
+{
+    if (!amax || K <= 0 || max_o < 0 || (max_o > 0 && !idx)) return -1;
+    int64_t n = 0;
+    for (int64_t j = 0; j < K; ++j)
+        if (amax[j] >= threshold) {
+            if (n < max_o) idx[n] = (int32_t)j;
+            ++n;
+        }
+    return n;
+}
+
+/* IEEE binary16 value nearest to v (ties to even), as a double; overflow
+ * goes to infinity, values below the subnormal range to zero. */
+static double fp16_round(float v)
+{
+    double a = fabs((double)v);
+    if (a == 0.0 || v != v) return (double)v;
+    double r;
+    if (a >= 65520.0) {                 /* at or past the midpoint above 65504 */
+        r = INFINITY;
+    } else {
+        int e;
+        frexp(a, &e);                   /* a = m * 2^e, m in [0.5, 1) */
+        int q = e - 11;                 /* spacing 2^(e-11) for normal halves */
+        if (q < -24) q = -24;           /* subnormal spacing 2^-24 */
+        double step = ldexp(1.0, q);
+        r = nearbyint(a / step) * step; /* exact quotient; default mode is to nearest even */
+    }
+    return v < 0 ? -r : r;
+}
+
+/* [TS36] §1.1 the FP16 part of the decomposition, reading R16:
+ * out[t, o] = sum over the first min(cnt, max) listed columns j of
+ * fp16(a[t, j]) * fp16(W[o, j]), exact products summed in double. */
+int zqo_outlier_product(const float* a, int64_t T, int64_t K, const float* W, int64_t N,
+                        const int32_t* idx, int64_t cnt, double* out)
+{
+    if (!a || !W || !out || T <= 0 || K <= 0 || N <= 0 || cnt < 0 || (cnt > 0 && !idx)) return ZQO_EARG;
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t o = 0; o < N; ++o) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < cnt; ++k) {
+                int64_t j = idx[k];
+                acc += fp16_round(a[t * K + j]) * fp16_round(W[o * K + j]);
+            }
+            out[t * N + o] = acc;
+        }
+    return ZQO_OK;
+}
+
+/* The INT8 part dequantized with an extra addend before bias and activation
+ * (the decomposition's sum, reading R16): y = act(s_tok s_grp acc + add + b). */
+int zqo_dequant_add(const int32_t* acc, int64_t T, int64_t N, const float* s_tok, const float* s_grp,
+                    int64_t G, const double* add, const float* bias, int act, float* y)
+{
+    if (!acc || !s_tok || !s_grp || !y || T <= 0 || N <= 0 || G <= 0 || N % G != 0 ||
+        (act != 0 && act != 1))
+        return ZQO_EARG;
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t o = 0; o < N; ++o) {
+            double v = (double)s_tok[t] * (double)s_grp[o / G] * (double)acc[t * N + o];
+            if (add) v += add[t * N + o];
+            if (bias) v += (double)bias[o];
+            if (act == 1) v = gelu_d(v);
+            y[t * N + o] = (float)v;
+        }
     return ZQO_OK;
 }
