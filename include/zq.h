@@ -254,6 +254,44 @@ int zq_smooth_weights(const float* W, int64_t N, int64_t K, const float* amax, f
                       const float* gamma, const float* beta, float* W_out,
                       float* gamma_out, float* beta_out, float* s, void* stream);
 
+/* ---- LLM.int8() mixed-precision decomposition ----------------------------
+ * [TS36] §1.1 (LLM.int8()): the input columns holding a value above the
+ * threshold alpha (6.0 on the pages) form the outlier set O; X[:, O] and the
+ * matching weight columns are multiplied in FP16, the other columns run
+ * through the INT8 path, and the two results are added.  Here, for a linear
+ * fed by a LayerNorm:
+ *   1. zq_smooth_calibrate(x, gamma, beta) gives the per-column absmax of
+ *      the LayerNorm output over the batch (zero-filled amax first);
+ *   2. zq_llmint8_select picks O = {j : amax_j >= threshold}, the lowest
+ *      ZQ_LLMINT8_MAX_OUTLIERS of them, and writes gamma/beta with zeros on
+ *      those columns;
+ *   3. zq_ln_quant(x, gamma_m, beta_m) quantizes the other columns per token
+ *      (the decomposed columns become zero codes and do not set the scale);
+ *   4. zq_llmint8_outlier_act and zq_llmint8_outlier_weights gather the
+ *      decomposed columns of the LayerNorm output and of the fp32 weights as
+ *      fp16 (round to nearest even), [T, 8] and [N, 8], zeros past the count;
+ *   5. zq_w8a8_linear_llmint8 runs the W8A8 GEMM (weights group-quantized
+ *      offline over all columns) whose epilogue adds sum_k xo[t,k] wo[o,k]
+ *      (exact fp16 products, fp32 accumulation) before bias and activation.
+ * idx: int32 [ZQ_LLMINT8_MAX_OUTLIERS] device (-1 past the count);
+ * count: int32 [1] device, the total number of columns >= threshold (it may
+ * exceed ZQ_LLMINT8_MAX_OUTLIERS; only the first ones are decomposed).
+ * Constraints: K % 16 == 0, K <= ZQ_MAX_H; out_kind ZQ_OUT_F32 or ZQ_OUT_BF16.
+ * Errors: NULL, SHAPE, ALIGN, DTYPE, CUDA, DEVICE. */
+#define ZQ_LLMINT8_MAX_OUTLIERS 8
+int zq_llmint8_select(const float* amax, int64_t K, float threshold, const float* gamma,
+                      const float* beta, int32_t* idx, int32_t* count, float* gamma_m,
+                      float* beta_m, void* stream);
+int zq_llmint8_outlier_act(const void* x, int x_dtype, int64_t T, int64_t K, const float* gamma,
+                           const float* beta, float eps, const int32_t* idx, const int32_t* count,
+                           void* xo, void* stream);
+int zq_llmint8_outlier_weights(const float* W, int64_t N, int64_t K, const int32_t* idx,
+                               const int32_t* count, void* wo, void* stream);
+int zq_w8a8_linear_llmint8(const int8_t* xq, const float* s_tok, int64_t T, int64_t K,
+                           const int8_t* Wq, const float* s_grp, int64_t N, int64_t group_rows,
+                           const float* bias, int act, int out_kind, const void* xo, const void* wo,
+                           void* y, void* stream);
+
 /* ---- diagnostics ----------------------------------------------------------
  * zq_device_status: synchronizes `stream`, then reads and clears the device
  * flag that bounded waits set on expiry.  Returns ZQ_OK, ZQ_ERR_TIMEOUT or

@@ -240,6 +240,71 @@ int zq_quantize_weights(const float* W, int64_t N, int64_t K, int64_t group_rows
     return launch_quantize_weights(W, N, K, group_rows, Wq, s_grp, di, as_stream(stream));
 }
 
+int zq_llmint8_select(const float* amax, int64_t K, float threshold, const float* gamma, const float* beta,
+                      int32_t* idx, int32_t* count, float* gamma_m, float* beta_m, void* stream) {
+    if (!amax || !idx || !count || !gamma || !gamma_m || !beta_m) return ZQ_ERR_NULL;
+    if (K <= 0 || K % 16 != 0 || K > ZQ_MAX_H) return ZQ_ERR_SHAPE;
+    if (!aligned(amax, 4) || !aligned(idx, 4) || !aligned(count, 4) || !aligned(gamma, 4) || !aligned(gamma_m, 4) ||
+        !aligned(beta_m, 4) || (beta && !aligned(beta, 4)))
+        return ZQ_ERR_ALIGN;
+    DeviceInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    return launch_llmint8_select(amax, K, threshold, gamma, beta, idx, count, gamma_m, beta_m, as_stream(stream));
+}
+
+int zq_llmint8_outlier_act(const void* x, int x_dtype, int64_t T, int64_t K, const float* gamma, const float* beta,
+                           float eps, const int32_t* idx, const int32_t* count, void* xo, void* stream) {
+    if (!x || !gamma || !idx || !count || !xo) return ZQ_ERR_NULL;
+    if (x_dtype != ZQ_F32 && x_dtype != ZQ_BF16) return ZQ_ERR_DTYPE;
+    if (T <= 0 || K <= 0 || K % 16 != 0 || K > ZQ_MAX_H || T > ((int64_t)1 << 31)) return ZQ_ERR_SHAPE;
+    if (!aligned(x, 16) || !aligned(xo, 16) || !aligned(gamma, 4) || (beta && !aligned(beta, 4))) return ZQ_ERR_ALIGN;
+    DeviceInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    return launch_llmint8_outlier_act(x, x_dtype, T, K, gamma, beta, eps, idx, count, static_cast<uint16_t*>(xo),
+                                      as_stream(stream));
+}
+
+int zq_llmint8_outlier_weights(const float* W, int64_t N, int64_t K, const int32_t* idx, const int32_t* count,
+                               void* wo, void* stream) {
+    if (!W || !idx || !count || !wo) return ZQ_ERR_NULL;
+    if (N <= 0 || K <= 0 || K % 16 != 0 || N > ((int64_t)1 << 40) / K) return ZQ_ERR_SHAPE;
+    if (!aligned(W, 16) || !aligned(wo, 16)) return ZQ_ERR_ALIGN;
+    DeviceInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    return launch_llmint8_outlier_weights(W, N, K, idx, count, static_cast<uint16_t*>(wo), as_stream(stream));
+}
+
+int zq_w8a8_linear_llmint8(const int8_t* xq, const float* s_tok, int64_t T, int64_t K, const int8_t* Wq,
+                           const float* s_grp, int64_t N, int64_t group_rows, const float* bias, int act,
+                           int out_kind, const void* xo, const void* wo, void* y, void* stream) {
+    if (out_kind != ZQ_OUT_F32 && out_kind != ZQ_OUT_BF16) return ZQ_ERR_DTYPE;
+    if (!xo || !wo) return ZQ_ERR_NULL;
+    if (!aligned(xo, 16) || !aligned(wo, 16)) return ZQ_ERR_ALIGN;
+    int rc = check_linear(xq, s_tok, T, K, Wq, s_grp, N, group_rows, bias, act, out_kind, y, nullptr, nullptr, 0,
+                          true);
+    if (rc) return rc;
+    DeviceInfo di;
+    if ((rc = device_info(&di))) return rc;
+    LinearArgs a{};
+    a.xq = xq;
+    a.s_tok = s_tok;
+    a.T = T;
+    a.K = K;
+    a.Wq = Wq;
+    a.s_grp = s_grp;
+    a.N = N;
+    a.G = group_rows;
+    a.bias = bias;
+    a.act = act;
+    a.out_kind = out_kind;
+    a.y = y;
+    return launch_w8a8_gemm_outliers(a, static_cast<const uint16_t*>(xo), static_cast<const uint16_t*>(wo), di,
+                                     as_stream(stream));
+}
+
 int zq_smooth_calibrate(const void* x, int x_dtype, int64_t T, int64_t H, const float* gamma,
                         const float* beta, float eps, float* amax, void* stream) {
     if (!x || !amax) return ZQ_ERR_NULL;

@@ -70,6 +70,10 @@ struct Params {
     int act;
     int group_m;        // tile raster: groups of group_m row tiles sweep all column tiles
     int* status;
+    // LLM.int8() outlier part (OUTL kernels): fp16 [M, 8] activations and
+    // fp16 [N, 8] weights of the decomposed columns (zeros past the count)
+    const uint16_t* xo;
+    const uint16_t* wo;
 };
 
 // Tile index -> (row tile, column tile).  Tiles run in groups of GM row tiles:
@@ -106,12 +110,13 @@ __host__ __device__ constexpr size_t smem_bytes() {
            (EPI == EPI_I32 ? 0 : EPI == EPI_BF16 && !SWAP ? 1 : 2) * BN * sizeof(float);
 }
 
-template <int BN, int STAGES, bool SWAP, int EPI, int EW>
+template <int BN, int STAGES, bool SWAP, int EPI, int EW, bool OUTL = false>
 __global__ void __launch_bounds__(block_threads<EW>(), 1)
 w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmY, const Params p) {
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128 is 16..256 step 16");
     static_assert(EW % 4 == 0 && EW >= 4 && EW <= 16, "epilogue warps cover the 4 TMEM lane quarters");
+    static_assert(!OUTL || (!SWAP && (EPI == EPI_F32 || EPI == EPI_BF16)), "outlier part: fp32/bf16 tiles");
     constexpr int kEpiThreads = 32 * EW;
     constexpr int B_STAGE = BN * BK;
     // epilogue column chunk (16 for the swapped 32-token tile: 32 there spills
@@ -352,6 +357,17 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 const int gm = mt * BM + r;  // token row owned by this thread
                 const bool row_ok = gm < p.M;
                 float amax = 0.0f;
+                float xo[8];  // this token's outlier activations (OUTL)
+                if constexpr (OUTL) {
+                    uint4 u = make_uint4(0u, 0u, 0u, 0u);
+                    if (row_ok) u = __ldg(reinterpret_cast<const uint4*>(p.xo) + gm);
+                    const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        xo[2 * q] = half_lo(uw[q]);
+                        xo[2 * q + 1] = half_hi(uw[q]);
+                    }
+                }
                 const uint32_t t_row = tmem_base + (uint32_t)(b * BN) + ((uint32_t)(quarter * 32) << 16);
                 static_assert(SWAP || CW == 32, "non-swapped tiles are whole 32-column chunks");
 #pragma unroll 1
@@ -374,7 +390,29 @@ w8a8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         for (int j = 0; j < 32; ++j) w[j] = v[j];
                     } else {
                         uint64_t f[16];
-                        if (gelu) {
+                        if constexpr (OUTL) {
+                            // the chunk's outlier weight columns, transposed ([k][column])
+                            // into this warp's staging box once its previous store has read it
+                            uint4 u = make_uint4(0u, 0u, 0u, 0u);
+                            if (n0 + lane < p.N) u = __ldg(reinterpret_cast<const uint4*>(p.wo) + n0 + lane);
+                            if (lane == 0) bulk_wait_read_all();
+                            __syncwarp();
+                            float* box = reinterpret_cast<float*>(stg);
+                            const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                box[(2 * q) * 32 + lane] = half_lo(uw[q]);
+                                box[(2 * q + 1) * 32 + lane] = half_hi(uw[q]);
+                            }
+                            __syncwarp();
+                            if (gelu) {
+                                if (uni) dequant_chunk_lanes_outl<true, true>(v, row_scale, ca, cb, xo, box, f);
+                                else dequant_chunk_lanes_outl<true, false>(v, row_scale, ca, cb, xo, box, f);
+                            } else {
+                                if (uni) dequant_chunk_lanes_outl<false, true>(v, row_scale, ca, cb, xo, box, f);
+                                else dequant_chunk_lanes_outl<false, false>(v, row_scale, ca, cb, xo, box, f);
+                            }
+                        } else if (gelu) {
                             if (uni) dequant_chunk_lanes<true, true>(v, row_scale, ca, cb, f);
                             else dequant_chunk_lanes<true, false>(v, row_scale, ca, cb, f);
                         } else {
@@ -588,13 +626,13 @@ int max_clusters(K kern, int S, size_t smem, int threads, int dev) {
     return cache[dev][S];
 }
 
-template <int BN, int STAGES, bool SWAP, int EPI, int EW>
+template <int BN, int STAGES, bool SWAP, int EPI, int EW, bool OUTL = false>
 int launch_cfg(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ty, const Params& p,
                const DeviceInfo& di, cudaStream_t st) {
     constexpr size_t kSmem = smem_bytes<BN, STAGES, SWAP, EPI, EW>();
     static_assert(kSmem <= 232448, "shared memory budget");
     static_assert(kSmem > 116 * 1024, "one CTA per SM (TMEM ownership)");
-    auto kern = w8a8_gemm_kernel<BN, STAGES, SWAP, EPI, EW>;
+    auto kern = w8a8_gemm_kernel<BN, STAGES, SWAP, EPI, EW, OUTL>;
     static bool attr_set[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -805,6 +843,43 @@ int launch_w8a8_gemm(const LinearArgs& a, const DeviceInfo& di, cudaStream_t st)
     if (bn == 256) return launch_epi<256, false>(epi, ta, tb, ty, p, di, st);
     if (bn == 192) return launch_epi<192, false>(epi, ta, tb, ty, p, di, st);
     return launch_epi<128, false>(epi, ta, tb, ty, p, di, st);
+}
+
+// LLM.int8() linear: the W8A8 GEMM whose epilogue adds the fp16 outlier
+// product before bias and activation (always the non-swapped kernel, 128-wide
+// tiles; fp32 or bf16 output).
+int launch_w8a8_gemm_outliers(const LinearArgs& a, const uint16_t* xo, const uint16_t* wo, const DeviceInfo& di,
+                              cudaStream_t st) {
+    const int epi = a.out_kind == ZQ_OUT_F32 ? EPI_F32 : EPI_BF16;
+    Params p{};
+    p.M = (int)a.T;
+    p.N = (int)a.N;
+    p.K = (int)a.K;
+    p.G = (int)a.G;
+    p.ldy = (int)a.N;
+    p.s_tok = a.s_tok;
+    p.s_grp = a.s_grp;
+    p.bias = a.bias;
+    p.y = a.y;
+    p.act = a.act;
+    p.status = di.status_word;
+    p.xo = xo;
+    p.wo = wo;
+    const int64_t m_tiles = (a.T + BM - 1) / BM;
+    int64_t gm = (24ll << 20) / ((int64_t)BM * a.K);
+    const int64_t n_tiles = (a.N + 127) / 128;
+    const int64_t min_gm = (di.sm_count + n_tiles - 1) / n_tiles;
+    if (gm < min_gm) gm = min_gm;
+    if (gm < 1) gm = 1;
+    p.group_m = (int)(gm < m_tiles ? gm : m_tiles);
+    CUtensorMap ta, tb, ty;
+    int rc;
+    if ((rc = make_tmap_i8(&ta, a.xq, a.T, a.K, BM))) return rc;
+    if ((rc = make_tmap_i8(&tb, a.Wq, a.N, a.K, 128))) return rc;
+    if ((rc = make_tmap_out(&ty, a.y, a.T, a.N, epi == EPI_BF16 ? 2 : 4))) return rc;
+    if (epi == EPI_F32)
+        return launch_cfg<128, stages_for<128, false, EPI_F32>(), false, EPI_F32, 16, true>(ta, tb, ty, p, di, st);
+    return launch_cfg<128, stages_for<128, false, EPI_BF16>(), false, EPI_BF16, 16, true>(ta, tb, ty, p, di, st);
 }
 
 }  // namespace zq

@@ -309,6 +309,43 @@ __device__ __forceinline__ void dequant_chunk_lanes(uint32_t (&v)[32], float row
     }
 }
 
+// fp16 halves of a 32-bit word (low half first), as floats.
+__device__ __forceinline__ float half_lo(uint32_t w) {
+    float f;
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.f32.f16 %0, lo;\n\t}" : "=f"(f) : "r"(w));
+    return f;
+}
+__device__ __forceinline__ float half_hi(uint32_t w) {
+    float f;
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.f32.f16 %0, hi;\n\t}" : "=f"(f) : "r"(w));
+    return f;
+}
+
+// dequant_chunk_lanes plus the LLM.int8() outlier part: before bias and
+// activation each column gains sum_k xo[k] * wo[column][k] (the decomposed
+// columns' fp16 values, exact products accumulated in fp32); the warp's
+// outlier weights sit transposed in shared memory, box[k * 32 + column].
+template <bool GELU, bool UNI>
+__device__ __forceinline__ void dequant_chunk_lanes_outl(uint32_t (&v)[32], float row_scale, float ca, float cb,
+                                                         const float (&xo)[8], const float* box, uint64_t (&f)[16]) {
+    acc32_to_f2(v, f);
+    const uint64_t rs2 = f2_splat(row_scale);
+    const uint64_t a_uni = f2_splat(row_scale * __shfl_sync(0xFFFFFFFFu, ca, 0));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const uint64_t a2 = UNI ? a_uni
+                                : f2_mul(rs2, f2_pack(__shfl_sync(0xFFFFFFFFu, ca, 2 * i),
+                                                      __shfl_sync(0xFFFFFFFFu, ca, 2 * i + 1)));
+        uint64_t o2 = f2_pack(__shfl_sync(0xFFFFFFFFu, cb, 2 * i), __shfl_sync(0xFFFFFFFFu, cb, 2 * i + 1));
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            o2 = f2_fma(f2_splat(xo[k]), *reinterpret_cast<const uint64_t*>(box + k * 32 + 2 * i), o2);
+        uint64_t t = f2_fma(a2, f[i], o2);
+        if (GELU) t = gelu2(t);
+        f[i] = t;
+    }
+}
+
 // Codes of four fp32 values packed little-endian into one word.
 // t = fl(y * inv) as a packed multiply; then fl(t + 1.5*2^23) (a scalar add
 // with explicit round-to-nearest, which is never contracted with the multiply)
@@ -627,6 +664,13 @@ int launch_rowq_pipe(const void* x, int x_dtype, int64_t T, int64_t H, bool ln, 
                      float* s_tok, const DeviceInfo& di, cudaStream_t st);
 int launch_requant_rows(const float* h, int64_t T, int64_t N, const uint32_t* amax_bits, int8_t* q,
                         float* s_tok, const DeviceInfo& di, cudaStream_t st);
+int launch_llmint8_select(const float* amax, int64_t K, float threshold, const float* gamma, const float* beta,
+                          int32_t* idx, int32_t* count, float* gamma_m, float* beta_m, cudaStream_t st);
+int launch_llmint8_outlier_act(const void* x, int x_dtype, int64_t T, int64_t K, const float* gamma,
+                               const float* beta, float eps, const int32_t* idx, const int32_t* count, uint16_t* xo,
+                               cudaStream_t st);
+int launch_llmint8_outlier_weights(const float* W, int64_t N, int64_t K, const int32_t* idx, const int32_t* count,
+                                   uint16_t* wo, cudaStream_t st);
 int launch_smooth_calibrate(const void* x, int x_dtype, int64_t T, int64_t H, const float* gamma,
                             const float* beta, float eps, float* amax, const DeviceInfo& di, cudaStream_t st);
 int launch_smooth_weights(const float* W, int64_t N, int64_t K, const float* amax, float alpha, const float* gamma,
@@ -648,6 +692,8 @@ struct LinearArgs {
     uint32_t* amax_ws;  // REQUANT (scratch path): [T] absmax bit patterns
 };
 int launch_w8a8_gemm(const LinearArgs& a, const DeviceInfo& di, cudaStream_t st);
+int launch_w8a8_gemm_outliers(const LinearArgs& a, const uint16_t* xo, const uint16_t* wo, const DeviceInfo& di,
+                              cudaStream_t st);
 // Requantizing linear with the per-token absmax exchanged between the CTAs of
 // a thread-block cluster (no scratch).  ZQ_ERR_SHAPE: shape not covered (the
 // caller then uses the scratch path).

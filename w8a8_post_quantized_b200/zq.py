@@ -34,8 +34,10 @@ EXPORTED = (
     "zq_w8a8_linear", "zq_linear_block_workspace", "zq_linear_block", "zq_device_status",
     "zq_status_string", "zq_last_cuda_error", "zq_version", "zq_launch_count",
     "zq_w8a8_linear_requant_noalloc", "zq_smooth_calibrate", "zq_smooth_weights",
-    "zq_watchdog_selftest",
+    "zq_watchdog_selftest", "zq_llmint8_select", "zq_llmint8_outlier_act", "zq_llmint8_outlier_weights",
+    "zq_w8a8_linear_llmint8",
 )
+ZQ_LLMINT8_MAX_OUTLIERS = 8
 
 
 class ZQError(RuntimeError):
@@ -77,6 +79,10 @@ def lib() -> ctypes.CDLL:
         "zq_smooth_calibrate": (I, [P, I, I64, I64, P, P, F, P, P]),
         "zq_smooth_weights": (I, [P, I64, I64, P, F, P, P, P, P, P, P, P]),
         "zq_watchdog_selftest": (I, [P]),
+        "zq_llmint8_select": (I, [P, I64, F, P, P, P, P, P, P, P]),
+        "zq_llmint8_outlier_act": (I, [P, I, I64, I64, P, P, F, P, P, P, P]),
+        "zq_llmint8_outlier_weights": (I, [P, I64, I64, P, P, P, P]),
+        "zq_w8a8_linear_llmint8": (I, [P, P, I64, I64, P, P, I64, I64, P, I, I, P, P, P, P]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -159,6 +165,50 @@ def zq_smooth_weights(W, amax, alpha=0.5, gamma=None, beta=None, W_out=None, gam
                                    _p(W_out), _p(gamma_out), _p(beta_out), _p(s), _s(stream)),
            "zq_smooth_weights")
     return W_out, gamma_out, beta_out, s
+
+
+def zq_llmint8_select(amax, gamma, beta=None, threshold=6.0, stream=None):
+    """LLM.int8() outlier columns: returns (idx [8] int32, count [1] int32,
+    gamma and beta zeroed on the decomposed columns)."""
+    K = amax.numel()
+    dev = amax.device
+    idx = torch.empty(ZQ_LLMINT8_MAX_OUTLIERS, dtype=torch.int32, device=dev)
+    count = torch.empty(1, dtype=torch.int32, device=dev)
+    gm = torch.empty(K, dtype=torch.float32, device=dev)
+    bm = torch.empty(K, dtype=torch.float32, device=dev)
+    _check(lib().zq_llmint8_select(_p(amax), K, float(threshold), _p(gamma), _p(beta), _p(idx), _p(count),
+                                   _p(gm), _p(bm), _s(stream)), "zq_llmint8_select")
+    return idx, count, gm, bm
+
+
+def zq_llmint8_outlier_act(x, gamma, beta, eps, idx, count, stream=None):
+    """The decomposed columns of LayerNorm(x) as fp16 [T, 8]."""
+    T, K = x.shape
+    xo = torch.empty((T, ZQ_LLMINT8_MAX_OUTLIERS), dtype=torch.float16, device=x.device)
+    _check(lib().zq_llmint8_outlier_act(_p(x), _dtype_code(x), T, K, _p(gamma), _p(beta), float(eps), _p(idx),
+                                        _p(count), _p(xo), _s(stream)), "zq_llmint8_outlier_act")
+    return xo
+
+
+def zq_llmint8_outlier_weights(W, idx, count, stream=None):
+    """The decomposed columns of the fp32 weights as fp16 [N, 8]."""
+    N, K = W.shape
+    wo = torch.empty((N, ZQ_LLMINT8_MAX_OUTLIERS), dtype=torch.float16, device=W.device)
+    _check(lib().zq_llmint8_outlier_weights(_p(W), N, K, _p(idx), _p(count), _p(wo), _s(stream)),
+           "zq_llmint8_outlier_weights")
+    return wo
+
+
+def zq_w8a8_linear_llmint8(xq, s_tok, Wq, s_grp, group_rows, xo, wo, bias=None, act=ZQ_ACT_NONE,
+                           out_kind=ZQ_OUT_BF16, y=None, stream=None):
+    """W8A8 linear plus the fp16 outlier product (before bias and activation)."""
+    T, K = xq.shape
+    N = Wq.shape[0]
+    y = torch.empty((T, N), dtype=_out_dtype(out_kind), device=xq.device) if y is None else y
+    _check(lib().zq_w8a8_linear_llmint8(_p(xq), _p(s_tok), T, K, _p(Wq), _p(s_grp), N, group_rows, _p(bias),
+                                        int(act), int(out_kind), _p(xo), _p(wo), _p(y), _s(stream)),
+           "zq_w8a8_linear_llmint8")
+    return y
 
 
 def zq_act_quant(x, bias=None, act=ZQ_ACT_NONE, q=None, s_tok=None, stream=None):
