@@ -230,10 +230,73 @@ def build_smooth_workload(W, zq, torch, device):
     return W
 
 
+def build_llmint8_workload(W, zq, torch, device):
+    """LLM.int8() decomposition on the BERT-base FFN's first linear, per batch:
+    column absmax of the LayerNorm output, outlier selection (alpha = 6) with
+    masked LayerNorm parameters, LN + token quant of the other columns, the
+    fp16 outlier operands, and the W8A8 GEMM whose epilogue adds the outlier
+    product (+ bias + GeLU, bf16 out)."""
+    w = inputs.bert_ffn()
+    lin = w.layers[0]
+    x = W.dev_act(w.x)
+    T, H = x.shape
+    g, b = W.dev(w.gamma), W.dev(w.beta)
+    W1 = W.dev(lin.W)
+    N = W1.shape[0]
+    G = lin.group_rows
+    Wq, sg = zq.zq_quantize_weights(W1, G)
+    bias = W.dev(lin.bias)
+    amax = torch.zeros(H, dtype=torch.float32, device=device)
+    idx = torch.empty(zq.ZQ_LLMINT8_MAX_OUTLIERS, dtype=torch.int32, device=device)
+    count = torch.empty(1, dtype=torch.int32, device=device)
+    gm, bm = torch.empty_like(g), torch.empty_like(b)
+    q = torch.empty((T, H), dtype=torch.int8, device=device)
+    st = torch.empty(T, dtype=torch.float32, device=device)
+    xo = torch.empty((T, zq.ZQ_LLMINT8_MAX_OUTLIERS), dtype=torch.float16, device=device)
+    wo = torch.empty((N, zq.ZQ_LLMINT8_MAX_OUTLIERS), dtype=torch.float16, device=device)
+    y = torch.empty((T, N), dtype=torch.bfloat16, device=device)
+    P = zq.lib()
+
+    def detect():
+        # the per-batch column absmax is a running max: restart it from zero
+        amax.zero_()
+        zq.zq_smooth_calibrate(x, g, b, w.eps, amax=amax)
+        zq._check(P.zq_llmint8_select(zq._p(amax), H, 6.0, zq._p(g), zq._p(b), zq._p(idx), zq._p(count),
+                                      zq._p(gm), zq._p(bm), zq._s(None)), "zq_llmint8_select")
+
+    def operands():
+        zq.zq_ln_quant(x, gm, bm, w.eps, q=q, s_tok=st)
+        zq._check(P.zq_llmint8_outlier_act(zq._p(x), zq._dtype_code(x), T, H, zq._p(g), zq._p(b), float(w.eps),
+                                           zq._p(idx), zq._p(count), zq._p(xo), zq._s(None)),
+                  "zq_llmint8_outlier_act")
+        zq._check(P.zq_llmint8_outlier_weights(zq._p(W1), N, H, zq._p(idx), zq._p(count), zq._p(wo), zq._s(None)),
+                  "zq_llmint8_outlier_weights")
+
+    W.stages.append(("detect", detect))
+    W.stages.append(("operands", operands))
+    W.stages.append(("linear1", lambda: zq.zq_w8a8_linear_llmint8(q, st, Wq, sg, G, xo, wo, bias=bias, act=1,
+                                                                   out_kind=zq.ZQ_OUT_BF16, y=y)))
+    xbytes = x.numel() * x.element_size()
+    W.kernel_units["detect"] = ("hbm", xbytes + 8 * H + 4 * H, "bytes")
+    W.kernel_units["operands"] = ("hbm", 2 * xbytes + T * H + 4 * T + 16 * T + 16 * N, "bytes")
+    ops = 2 * T * N * H + 2 * T * N * zq.ZQ_LLMINT8_MAX_OUTLIERS
+    W.kernel_units["linear1"] = ("tensor", ops, "ops")
+    W.ops = 2 * T * N * H
+    W.tokens = T
+    W.h2d_src = x
+    W.out = y
+    W.config = {"workload": "bert_ffn W1 with LLM.int8() decomposition (alpha 6, up to 8 fp16 columns)",
+                "tokens": T, "hidden": H, "x_dtype": w.x.dtype, "epilogue": "fp16 outliers + bias + gelu",
+                "out_dtype": "bf16"}
+    return W
+
+
 def build_workload(name, zq, torch, device):
     W = Workload(name, zq, torch, device)
     if name == "bert_smooth":
         return build_smooth_workload(W, zq, torch, device)
+    if name == "bert_llmint8":
+        return build_llmint8_workload(W, zq, torch, device)
     if name in ("bert_ffn", "gptj_qkv", "tiny"):
         w = {"bert_ffn": inputs.bert_ffn, "gptj_qkv": inputs.gptj_qkv, "tiny": inputs.tiny}[name]()
     elif name == "neox_decode":
@@ -480,6 +543,8 @@ def oracle_sample(name, budget_s=12.0, max_rows=None):
         w = inputs.gemm_sweep_point(M, inputs.GEMM_SWEEP_M.index(M))
     elif name == "bert_smooth":
         return oracle_smooth_sample(budget_s, max_rows)
+    elif name == "bert_llmint8":
+        return oracle_llmint8_sample(budget_s, max_rows)
     else:
         raise SystemExit(f"no oracle baseline for {name}")
     qlayers = [(*oracle.quantize_weights(l.W, l.group_rows), l.bias, l.group_rows) for l in w.layers]
@@ -533,6 +598,28 @@ def oracle_smooth_sample(budget_s=12.0, max_rows=None):
     t_total += time.perf_counter() - t0
     nbytes += 8 * N * H + 16 * H
     return nbytes, t_total, rows_done, T
+
+
+def oracle_llmint8_sample(budget_s=12.0, max_rows=None):
+    """The oracle's LLM.int8() layer (BERT W1, GeLU) on row chunks of the BERT
+    batch (outliers detected on each chunk).  Returns (ops, seconds, rows, T)."""
+    import oracle
+    w = inputs.bert_ffn()
+    lin = w.layers[0]
+    Wq, sg = oracle.quantize_weights(lin.W, lin.group_rows)
+    T, H = w.x.f32.shape
+    N = lin.W.shape[0]
+    rows_done, ops, t_total = 0, 0, 0.0
+    limit = max_rows if max_rows is not None else T
+    while rows_done < limit and t_total < budget_s:
+        x = w.x.f32[rows_done % T:rows_done % T + 8]
+        t0 = time.perf_counter()
+        oracle.int8_decomposed_ln_linear(x, w.gamma, w.beta, w.eps, lin.W, Wq, sg, lin.group_rows, lin.bias,
+                                         oracle.ACT_GELU)
+        t_total += time.perf_counter() - t0
+        rows_done += x.shape[0]
+        ops += 2 * x.shape[0] * N * H
+    return ops, t_total, rows_done, T
 
 
 # -------------------------------------------------------------------- main
