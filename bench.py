@@ -497,13 +497,18 @@ def count_launches(W, zq, torch):
     return sum(per_stage.values()), per_stage
 
 
+# The sources of the hot-path kernels the ncu records describe (the
+# quantizers, both GEMMs, their shared helpers and their launch code).
+PROFILED_SOURCES = ("zq_internal.cuh", "zq_api.cu", "zq_rowquant.cu", "zq_quant.cu", "zq_gemm.cu",
+                    "zq_gemm_creq.cu")
+
+
 def kernel_source_hash():
-    """Hash of the CUDA sources: ncu counters recorded for another version of
-    the kernels are not reported."""
-    import glob
+    """Hash of the hot-path kernel sources: ncu counters recorded for another
+    version of those kernels are not reported."""
     import hashlib
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "w8a8_post_quantized_b200", "csrc", "*.cu*"))):
+    for f in sorted(os.path.join(ROOT, "w8a8_post_quantized_b200", "csrc", n) for n in PROFILED_SOURCES):
         with open(f, "rb") as fh:
             h.update(os.path.basename(f).encode())
             h.update(fh.read())
