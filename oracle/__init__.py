@@ -17,10 +17,12 @@ Sources (web pages):
   [SQ]   "SmoothQuant技术解析：大模型INT8量化的突破与实践" §2.2, §3 and [TS36]
          §1.3 -- per-channel smoothing folded offline into the weights.
   [TS36] §1.1 LLM.int8() -- mixed-precision decomposition of outlier columns.
+  [ZQ], [TS36] §1.2.2 group-wise paragraph read along the input axis
+         (reading R17 of zq_oracle.c) -- K-axis weight groups.
 
-Every function here is pinned by ``tests/test_oracle_pins.py`` against
-hand-worked examples (``tests/golden/``), closed forms, invariants and
-library routines; none is "parity unpinned".
+Every function here is pinned by the ``tests/test_oracle_*.py`` files
+against hand-worked examples (``tests/golden/``), closed forms, invariants
+and library routines; none is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -73,6 +75,8 @@ def _L():
             "zqo_smooth_fold": [P, I64, I64, P, P, P, P, P, P],
             "zqo_outlier_product": [P, I64, I64, P, I64, P, I64, P],
             "zqo_dequant_add": [P, I64, I64, P, P, I64, P, P, ctypes.c_int, P],
+            "zqo_quantize_weights_kgroups": [P, I64, I64, I64, P, P],
+            "zqo_linear_kgroups": [P, I64, I64, P, I64, I64, P, P, P, ctypes.c_int, P],
         }
         for name, args in sig.items():
             fn = getattr(lib, name)
@@ -335,3 +339,45 @@ def int8_decomposed_ln_linear(x, gamma, beta, eps, W, Wq, s_grp, group_rows, bia
     add = outlier_product(a, W, idx)
     y = dequant_add(gemm_i32(xq, Wq), st, s_grp, group_rows, add, bias, act)
     return y, idx, n
+
+
+# ---- K-axis weight groups ([ZQ], [TS36] §1.2.2, reading R17) ---------------
+
+def quantize_weights_kgroups(W, group_cols):
+    """Group-wise weight quantization along the input axis: W fp32 [N, K] ->
+    (Wq int8 [N, K], s_w fp32 [N, K / group_cols]); group (o, j) is row o,
+    columns j*group_cols .. (j+1)*group_cols - 1."""
+    W, pw = _c(W, np.float32)
+    N, K = W.shape
+    Wq = np.empty((N, K), np.int8)
+    s = np.empty((N, K // group_cols if group_cols > 0 else 0), np.float32)
+    _chk(_L().zqo_quantize_weights_kgroups(pw, N, K, group_cols, Wq.ctypes.data, s.ctypes.data),
+         "quantize_weights_kgroups")
+    return Wq, s
+
+
+def linear_kgroups(xq, s_tok, Wq, s_w, group_cols, bias=None, act=ACT_NONE):
+    """y = act(s_tok[t] * sum_j s_w[o, j] * acc_j[t, o] + bias[o]) in double -> fp32,
+    acc_j the exact integer product over the columns of group j."""
+    xq, px = _c(xq, np.int8)
+    Wq, pw = _c(Wq, np.int8)
+    st, ps = _c(s_tok, np.float32)
+    sw, pg = _c(s_w, np.float32)
+    T, K = xq.shape
+    N, K2 = Wq.shape
+    if K != K2 or sw.shape != (N, K // group_cols):
+        raise OracleError("linear_kgroups: shape mismatch")
+    pb = None
+    if bias is not None:
+        bias, pb = _c(bias, np.float32)
+    y = np.empty((T, N), np.float32)
+    _chk(_L().zqo_linear_kgroups(px, T, K, pw, N, group_cols, ps, pg, pb, int(act), y.ctypes.data),
+         "linear_kgroups")
+    return y
+
+
+def ln_linear_kgroups(x, gamma, beta, eps, Wq, s_w, group_cols, bias=None, act=ACT_NONE):
+    """LN + per-token quantization, then the K-group linear (fp32 out)."""
+    xq, st = ln_quant(x, gamma, beta, eps)
+    return linear_kgroups(xq, st, Wq, s_w, group_cols, bias, act)
+

@@ -68,6 +68,13 @@
  *      the outlier operands are rounded to fp16 (round to nearest even) and
  *      multiplied exactly; the outlier product is added to the dequantized
  *      INT8 result before bias and activation.
+ *  R17 K-axis weight groups (the other reading of the group-wise paragraph
+ *      of [ZQ] and [TS36] §1.2.2, which split W into groups without naming
+ *      the axis): a group is one output row o and Gk consecutive input
+ *      columns j*Gk .. j*Gk+Gk-1, quantized as one span with scale
+ *      s_w[o, j].  The linear then takes each group's exact integer
+ *      partial product, scales it by s_w[o, j], sums over j, multiplies by
+ *      the token scale and adds bias (all in double, one rounding to fp32).
  *
  * Status codes: 0 = ok, 1 = bad argument, 2 = int32 overflow in the GEMM.
  */
@@ -349,6 +356,50 @@ int zqo_dequant_add(const int32_t* acc, int64_t T, int64_t N, const float* s_tok
         for (int64_t o = 0; o < N; ++o) {
             double v = (double)s_tok[t] * (double)s_grp[o / G] * (double)acc[t * N + o];
             if (add) v += add[t * N + o];
+            if (bias) v += (double)bias[o];
+            if (act == 1) v = gelu_d(v);
+            y[t * N + o] = (float)v;
+        }
+    return ZQO_OK;
+}
+
+/* [ZQ] group-wise weight quantization along the input axis, reading R17.
+ * W is [N, K] row-major; group (o, j) is W[o, j*Gk .. j*Gk+Gk-1], quantized
+ * as one span.  Wq is [N, K]; s_w is [N, K/Gk] row-major. */
+int zqo_quantize_weights_kgroups(const float* W, int64_t N, int64_t K, int64_t Gk, int8_t* Wq,
+                                 float* s_w)
+{
+    if (!W || !Wq || !s_w || N <= 0 || K <= 0 || Gk <= 0 || K % Gk != 0) return ZQO_EARG;
+    const int64_t ng = K / Gk;
+    for (int64_t o = 0; o < N; ++o)
+        for (int64_t j = 0; j < ng; ++j) {
+            int rc = zqo_quantize_span(W + o * K + j * Gk, Gk, Wq + o * K + j * Gk, &s_w[o * ng + j]);
+            if (rc) return rc;
+        }
+    return ZQO_OK;
+}
+
+/* The W8A8 linear with K-axis weight groups (reading R17; the dequantization
+ * of [TS36] §1.2.2 applied per group, bias per reading R8):
+ *   acc_j[t, o] = sum over k in group j of xq[t, k] * Wq[o, k]   (exact)
+ *   y[t, o] = act(s_tok[t] * sum_j s_w[o, j] * acc_j[t, o] + bias[o]). */
+int zqo_linear_kgroups(const int8_t* xq, int64_t T, int64_t K, const int8_t* Wq, int64_t N, int64_t Gk,
+                       const float* s_tok, const float* s_w, const float* bias, int act, float* y)
+{
+    if (!xq || !Wq || !s_tok || !s_w || !y || T <= 0 || K <= 0 || N <= 0 || Gk <= 0 || K % Gk != 0 ||
+        (act != 0 && act != 1))
+        return ZQO_EARG;
+    const int64_t ng = K / Gk;
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t o = 0; o < N; ++o) {
+            double v = 0.0;
+            for (int64_t j = 0; j < ng; ++j) {
+                int64_t acc = 0;
+                for (int64_t k = j * Gk; k < (j + 1) * Gk; ++k)
+                    acc += (int64_t)xq[t * K + k] * (int64_t)Wq[o * K + k];
+                v += (double)s_w[o * ng + j] * (double)acc;
+            }
+            v *= (double)s_tok[t];
             if (bias) v += (double)bias[o];
             if (act == 1) v = gelu_d(v);
             y[t * N + o] = (float)v;
