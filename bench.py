@@ -291,8 +291,47 @@ def build_llmint8_workload(W, zq, torch, device):
     return W
 
 
+KGROUP_COLS = 128
+
+
+def build_kgroup_workload(W, zq, torch, device):
+    """The GPT-J-6B QKV projection (2048 tokens, 4096 -> 12288, bf16 out) with
+    K-axis weight groups: LN + token quant, then the INT8 GEMM whose epilogue
+    scales every 128-column group's partial product as it completes."""
+    w = inputs.gptj_qkv()
+    lin = w.layers[0]
+    x = W.dev_act(w.x)
+    T, K = x.shape
+    N = lin.W.shape[0]
+    G = KGROUP_COLS
+    g, b = W.dev(w.gamma), W.dev(w.beta)
+    q1 = torch.empty((T, K), dtype=torch.int8, device=device)
+    st1 = torch.empty(T, dtype=torch.float32, device=device)
+    Wq, sw = zq.zq_quantize_weights_kgroups(W.dev(lin.W), G)
+    bias = W.dev(lin.bias)
+    y = torch.empty((T, N), dtype=torch.bfloat16, device=device)
+    torch.cuda.synchronize()
+    W.stages.append(("ln_quant", lambda: zq.zq_ln_quant(x, g, b, w.eps, q=q1, s_tok=st1)))
+    W.stages.append(("linear1", lambda: zq.zq_w8a8_linear_kgroups(q1, st1, Wq, sw, G, bias=bias,
+                                                                   out_kind=zq.ZQ_OUT_BF16, y=y)))
+    xbytes = x.numel() * x.element_size()
+    W.kernel_units["ln_quant"] = ("hbm", xbytes + T * K + 4 * T + 8 * K, "bytes")
+    ops = 2 * T * N * K
+    W.kernel_units["linear1"] = ("tensor", ops, "ops")
+    W.ops = ops
+    W.tokens = T
+    W.h2d_src = x
+    W.out = y
+    W.config = {"workload": f"gptj_6b_qkv_{T}x{K}x{N}_kgroups{G}", "tokens": T, "hidden": K,
+                "x_dtype": w.x.dtype, "layers": [[N, K, G]], "weight_groups": f"{G} input columns per scale",
+                "epilogue": "per-group scale, bias", "out_dtype": "bf16"}
+    return W
+
+
 def build_workload(name, zq, torch, device):
     W = Workload(name, zq, torch, device)
+    if name == "gptj_qkv_kgroups":
+        return build_kgroup_workload(W, zq, torch, device)
     if name == "bert_smooth":
         return build_smooth_workload(W, zq, torch, device)
     if name == "bert_llmint8":
@@ -501,14 +540,16 @@ def count_launches(W, zq, torch):
 # quantizers, both GEMMs, their shared helpers and their launch code).
 PROFILED_SOURCES = ("zq_internal.cuh", "zq_api.cu", "zq_rowquant.cu", "zq_quant.cu", "zq_gemm.cu",
                     "zq_gemm_creq.cu")
+# ... and of the K-axis group linear (its kernel, helpers, tensor-map code)
+KGROUP_SOURCES = ("zq_internal.cuh", "zq_kgroup.cu", "zq_gemm.cu")
 
 
-def kernel_source_hash():
+def kernel_source_hash(sources=PROFILED_SOURCES):
     """Hash of the hot-path kernel sources: ncu counters recorded for another
     version of those kernels are not reported."""
     import hashlib
     h = hashlib.sha256()
-    for f in sorted(os.path.join(ROOT, "w8a8_post_quantized_b200", "csrc", n) for n in PROFILED_SOURCES):
+    for f in sorted(os.path.join(ROOT, "w8a8_post_quantized_b200", "csrc", n) for n in sources):
         with open(f, "rb") as fh:
             h.update(os.path.basename(f).encode())
             h.update(fh.read())
@@ -524,7 +565,8 @@ def recorded_traffic(workload, stage):
     with open(path) as f:
         d = json.load(f)
     e = d.get(f"{workload}:{stage}")
-    if not e or e.get("source_hash") != kernel_source_hash():
+    srcs = KGROUP_SOURCES if workload == "gptj_qkv_kgroups" and stage == "linear1" else PROFILED_SOURCES
+    if not e or e.get("source_hash") != kernel_source_hash(srcs):
         return None
     return e.get("dram_bytes")
 
@@ -550,6 +592,8 @@ def oracle_sample(name, budget_s=12.0, max_rows=None):
         return oracle_smooth_sample(budget_s, max_rows)
     elif name == "bert_llmint8":
         return oracle_llmint8_sample(budget_s, max_rows)
+    elif name == "gptj_qkv_kgroups":
+        return oracle_kgroup_sample(budget_s, max_rows)
     else:
         raise SystemExit(f"no oracle baseline for {name}")
     qlayers = [(*oracle.quantize_weights(l.W, l.group_rows), l.bias, l.group_rows) for l in w.layers]
@@ -624,6 +668,27 @@ def oracle_llmint8_sample(budget_s=12.0, max_rows=None):
         t_total += time.perf_counter() - t0
         rows_done += x.shape[0]
         ops += 2 * x.shape[0] * N * H
+    return ops, t_total, rows_done, T
+
+
+def oracle_kgroup_sample(budget_s=12.0, max_rows=None):
+    """The oracle's LN + token quant + K-group linear (GPT-J QKV, 128-column
+    groups) on row chunks.  Returns (ops, seconds, rows, T)."""
+    import oracle
+    w = inputs.gptj_qkv()
+    lin = w.layers[0]
+    Wq, sw = oracle.quantize_weights_kgroups(lin.W, KGROUP_COLS)
+    T, K = w.x.f32.shape
+    N = lin.W.shape[0]
+    rows_done, ops, t_total = 0, 0, 0.0
+    limit = max_rows if max_rows is not None else T
+    while rows_done < limit and t_total < budget_s:
+        x = w.x.f32[rows_done % T:rows_done % T + 4]
+        t0 = time.perf_counter()
+        oracle.ln_linear_kgroups(x, w.gamma, w.beta, w.eps, Wq, sw, KGROUP_COLS, lin.bias)
+        t_total += time.perf_counter() - t0
+        rows_done += x.shape[0]
+        ops += 2 * x.shape[0] * N * K
     return ops, t_total, rows_done, T
 
 

@@ -292,6 +292,39 @@ int zq_w8a8_linear_llmint8(const int8_t* xq, const float* s_tok, int64_t T, int6
                            const float* bias, int act, int out_kind, const void* xo, const void* wo,
                            void* y, void* stream);
 
+/* ---- K-axis weight groups ------------------------------------------------
+ * [ZQ] group-wise weight quantization and [TS36] §1.2.2 (group-wise weights;
+ * the INT32 accumulation scaled by the weight and activation scales), with
+ * the groups taken along the input axis: group (o, j) is output row o and
+ * the group_cols (Gk) consecutive input columns j*Gk .. j*Gk+Gk-1, with its
+ * own scale.  The scale then varies along the contraction, so the linear
+ * scales every group's exact INT32 partial product before summing:
+ *   y[t, o] = act(s_tok[t] * sum_j s_w[j, o] * acc_j[t, o] + bias[o]),
+ *   acc_j[t, o] = sum over k in group j of xq[t, k] * Wq[o, k].
+ * zq_quantize_weights_kgroups:
+ *   W   : fp32 [N, K] device, row-major.
+ *   Wq  : int8 [N, K] device (output): rint(w * (127/absmax)), ties to even,
+ *         clamped to [-127, 127]; an all-zero group gets zero codes.
+ *   s_w : fp32 [K/Gk, N] device (output), GROUP-MAJOR: s_w[j*N + o] is the
+ *         scale absmax/127 of group (o, j).
+ *   Constraints: K % 16 == 0, K % Gk == 0.  Errors: NULL, SHAPE, ALIGN, CUDA,
+ *   DEVICE.
+ * zq_w8a8_linear_kgroups:
+ *   xq, s_tok : int8 [T, K] and fp32 [T] device (from zq_ln_quant /
+ *         zq_act_quant); Wq, s_w as written above; bias fp32 [N] or NULL;
+ *   act ZQ_ACT_NONE or ZQ_ACT_GELU; out_kind ZQ_OUT_F32 or ZQ_OUT_BF16;
+ *   y : [T, N] device (output).  The group sums accumulate in fp32 in the
+ *   order j = 0, 1, ...; the token scale multiplies the sum, then bias.
+ *   Constraints: Gk % 32 == 0 (a tensor-core k-step of 32 INT8 values never
+ *   straddles a group), Gk <= 256 (|acc_j| <= 2^22, see the kernel), K % Gk
+ *   == 0, N % 16 == 0.  Alignment: xq, Wq, y, s_w and bias 16 bytes; s_tok 4.
+ *   Errors: NULL, SHAPE, ALIGN, DTYPE, CUDA, DEVICE. */
+int zq_quantize_weights_kgroups(const float* W, int64_t N, int64_t K, int64_t group_cols,
+                                int8_t* Wq, float* s_w, void* stream);
+int zq_w8a8_linear_kgroups(const int8_t* xq, const float* s_tok, int64_t T, int64_t K,
+                           const int8_t* Wq, const float* s_w, int64_t N, int64_t group_cols,
+                           const float* bias, int act, int out_kind, void* y, void* stream);
+
 /* ---- diagnostics ----------------------------------------------------------
  * zq_device_status: synchronizes `stream`, then reads and clears the device
  * flag that bounded waits set on expiry.  Returns ZQ_OK, ZQ_ERR_TIMEOUT or

@@ -35,7 +35,7 @@ EXPORTED = (
     "zq_status_string", "zq_last_cuda_error", "zq_version", "zq_launch_count",
     "zq_w8a8_linear_requant_noalloc", "zq_smooth_calibrate", "zq_smooth_weights",
     "zq_watchdog_selftest", "zq_llmint8_select", "zq_llmint8_outlier_act", "zq_llmint8_outlier_weights",
-    "zq_w8a8_linear_llmint8",
+    "zq_w8a8_linear_llmint8", "zq_quantize_weights_kgroups", "zq_w8a8_linear_kgroups",
 )
 ZQ_LLMINT8_MAX_OUTLIERS = 8
 
@@ -83,6 +83,8 @@ def lib() -> ctypes.CDLL:
         "zq_llmint8_outlier_act": (I, [P, I, I64, I64, P, P, F, P, P, P, P]),
         "zq_llmint8_outlier_weights": (I, [P, I64, I64, P, P, P, P]),
         "zq_w8a8_linear_llmint8": (I, [P, P, I64, I64, P, P, I64, I64, P, I, I, P, P, P, P]),
+        "zq_quantize_weights_kgroups": (I, [P, I64, I64, I64, P, P, P]),
+        "zq_w8a8_linear_kgroups": (I, [P, P, I64, I64, P, P, I64, I64, P, I, I, P, P]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -208,6 +210,30 @@ def zq_w8a8_linear_llmint8(xq, s_tok, Wq, s_grp, group_rows, xo, wo, bias=None, 
     _check(lib().zq_w8a8_linear_llmint8(_p(xq), _p(s_tok), T, K, _p(Wq), _p(s_grp), N, group_rows, _p(bias),
                                         int(act), int(out_kind), _p(xo), _p(wo), _p(y), _s(stream)),
            "zq_w8a8_linear_llmint8")
+    return y
+
+
+def zq_quantize_weights_kgroups(W, group_cols, Wq=None, s_w=None, stream=None):
+    """K-axis groups: returns Wq int8 [N, K] and the group-major scales s_w
+    fp32 [K / group_cols, N]."""
+    N, K = W.shape
+    Wq = torch.empty((N, K), dtype=torch.int8, device=W.device) if Wq is None else Wq
+    s_w = (torch.empty((K // max(group_cols, 1), N), dtype=torch.float32, device=W.device)
+           if s_w is None else s_w)
+    _check(lib().zq_quantize_weights_kgroups(_p(W), N, K, group_cols, _p(Wq), _p(s_w), _s(stream)),
+           "zq_quantize_weights_kgroups")
+    return Wq, s_w
+
+
+def zq_w8a8_linear_kgroups(xq, s_tok, Wq, s_w, group_cols, bias=None, act=ZQ_ACT_NONE,
+                           out_kind=ZQ_OUT_BF16, y=None, stream=None):
+    """W8A8 linear with K-axis weight groups (s_w group-major [K / group_cols, N])."""
+    T, K = xq.shape
+    N = Wq.shape[0]
+    y = torch.empty((T, N), dtype=_out_dtype(out_kind), device=xq.device) if y is None else y
+    _check(lib().zq_w8a8_linear_kgroups(_p(xq), _p(s_tok), T, K, _p(Wq), _p(s_w), N, group_cols, _p(bias),
+                                        int(act), int(out_kind), _p(y), _s(stream)),
+           "zq_w8a8_linear_kgroups")
     return y
 
 
