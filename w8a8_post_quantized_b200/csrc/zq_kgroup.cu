@@ -14,13 +14,17 @@
 // with s_w stored group-major ([K/Gk, N]) so one group's scales for a tile's
 // columns are contiguous.
 //
-// Structure (one persistent CTA per SM, 2 + EW warps, 128 x 128 tiles):
+// Structure (one persistent CTA per SM, 128 x 128 tiles, 12 warps in three
+// warpgroups; warpgroup 0 gives up registers to the epilogue with
+// setmaxnreg: 40 per thread there, 232 in warpgroups 1-2):
 //   warp 0   TMA producer: operand stages (128 rows x 128 bytes of each
 //            operand, 128-byte swizzle);
 //   warp 1   one thread issues tcgen05.mma kind::i8 (K = 32 each) into one of
 //            NSLOT TMEM accumulators -- one accumulator per group -- and
 //            commits the slot after the group's last k-step;
-//   warps 2+ epilogue: per group, tcgen05.ld of the slot, each value scaled
+//   warps 2-3 idle;
+//   warps 4-11 epilogue (two per TMEM lane quarter, 64 columns each): per
+//            group, one tcgen05.ld round trip for the slot, each value scaled
 //            by its column's group scale and added to fp32 running sums in
 //            registers; after a tile's last group: token scale, bias,
 //            optional GeLU, TMA store (fp32 or bf16).  Each warp fetches the
@@ -52,6 +56,13 @@ constexpr int KG_UK = 32;      // K per tcgen05.mma of kind::i8
 constexpr int KG_NSLOT = 4;    // TMEM accumulators: 4 x 128 columns = all of TMEM
 constexpr int KG_PF = 4;       // group scales fetched this many groups ahead
 constexpr int KG_RING = KG_PF + 1;
+constexpr int KG_EW = 8;                        // epilogue warps
+constexpr int KG_THREADS = 128 + 32 * KG_EW;    // warpgroup 0 + two epilogue warpgroups
+constexpr uint32_t KG_REG_LAUNCH = 168;         // registers per thread at launch (65536 / 384, rounded to 8)
+constexpr uint32_t KG_REG_LOW = 40;             // warpgroup 0 after setmaxnreg.dec
+constexpr uint32_t KG_REG_HIGH = 232;           // epilogue warpgroups after setmaxnreg.inc
+static_assert(128 * KG_REG_LOW + 256 * KG_REG_HIGH <= KG_THREADS * KG_REG_LAUNCH,
+              "the epilogue's registers come out of the block's launch allocation");
 constexpr int KG_A = KG_BM * KG_BK;
 constexpr int KG_B = KG_BN * KG_BK;
 constexpr uint32_t kMagicBits = 0x4B400000u;  // 1.5 * 2^23
@@ -119,10 +130,10 @@ __device__ __forceinline__ void kg_tile(int tile, int m_tiles, int n_tiles, int 
 }
 
 template <int EPI, int EW, int STAGES>
-__global__ void __launch_bounds__(64 + 32 * EW, 1)
+__global__ void __launch_bounds__(KG_THREADS, 1)
 w8a8_kgroup_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmY, const KgParams p) {
-    static_assert(EW == 4 || EW == 8, "epilogue warps cover the 4 TMEM lane quarters");
+    static_assert(EW == KG_EW, "two epilogue warpgroups");
     constexpr int SLICES = EW / 4;
     constexpr int COLS = KG_BN / SLICES;  // columns per epilogue warp
     constexpr int NCH = COLS / 32;        // 32-column chunks per epilogue warp
@@ -188,63 +199,68 @@ w8a8_kgroup_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     const int SPG = p.G / KG_UK;    // k-steps per group
     const int NG = p.K / p.G;       // groups per tile
 
-    if (warp == 0) {
-        // ------------------------------------------------ TMA producer
-        if (lane == 0) {
-            griddep_wait();  // the activation codes are the previous grid's output
-            uint32_t it = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-                int mt, nt;
-                kg_tile(tile, m_tiles, n_tiles, p.group_m, mt, nt);
-                const int n0 = nt * KG_BN;
-                for (int kb = 0; kb < kblocks; ++kb) {
-                    const int s = it % STAGES;
-                    const uint32_t ph = (it / STAGES) & 1u;
-                    if (!mbar_wait(bar_empty(s), ph ^ 1u, abort_flag, p.status, KG_SITE_PROD_EMPTY)) {
-                        ok = false;
-                        break;
+    if (warp < 4) {
+        // warpgroup 0 as a whole hands registers to the epilogue
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(KG_REG_LOW));
+        if (warp == 0) {
+            // ------------------------------------------------ TMA producer
+            if (lane == 0) {
+                griddep_wait();  // the activation codes are the previous grid's output
+                uint32_t it = 0;
+                bool ok = true;
+                for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+                    int mt, nt;
+                    kg_tile(tile, m_tiles, n_tiles, p.group_m, mt, nt);
+                    const int n0 = nt * KG_BN;
+                    for (int kb = 0; kb < kblocks; ++kb) {
+                        const int s = it % STAGES;
+                        const uint32_t ph = (it / STAGES) & 1u;
+                        if (!mbar_wait(bar_empty(s), ph ^ 1u, abort_flag, p.status, KG_SITE_PROD_EMPTY)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(bar_full(s), KG_A + KG_B);
+                        tma_load_2d(sA + s * KG_A, &tmA, bar_full(s), kb * KG_BK, mt * KG_BM);
+                        tma_load_2d(sB + s * KG_B, &tmB, bar_full(s), kb * KG_BK, n0);
+                        ++it;
                     }
-                    mbar_arrive_expect_tx(bar_full(s), KG_A + KG_B);
-                    tma_load_2d(sA + s * KG_A, &tmA, bar_full(s), kb * KG_BK, mt * KG_BM);
-                    tma_load_2d(sB + s * KG_B, &tmB, bar_full(s), kb * KG_BK, n0);
-                    ++it;
                 }
+                // every copy this thread issued lands before the CTA can exit
+                const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0u;
+                for (uint32_t j = first; j < it; ++j)
+                    mbar_wait(bar_full(j % STAGES), (j / STAGES) & 1u, nullptr, p.status, KG_SITE_DRAIN);
             }
-            // every copy this thread issued lands before the CTA can exit
-            const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0u;
-            for (uint32_t j = first; j < it; ++j)
-                mbar_wait(bar_full(j % STAGES), (j / STAGES) & 1u, nullptr, p.status, KG_SITE_DRAIN);
-        }
-        __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            // One thread issues everything, so the loop keeps to counters (no
-            // division): `left` = k-steps left in the current group.
-            uint32_t it = 0, gc = 0, d = tmem_base;
-            int left = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-                for (int kb = 0; kb < kblocks; ++kb, ++it) {
-                    const int s = it % STAGES;
-                    const uint32_t ph = (it / STAGES) & 1u;
-                    if (!mbar_wait(bar_full(s), ph, abort_flag, p.status, KG_SITE_MMA_FULL)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint64_t da = sdesc_k_sw128(sA + s * KG_A);
-                    const uint64_t db = sdesc_k_sw128(sB + s * KG_B);
-                    const int nk = min(4, KS - 4 * kb);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        if (k < nk && ok) {
+            __syncwarp();
+        } else if (warp == 1) {
+            // ------------------------------------------------ MMA issuer
+            if (lane == 0) {
+                // One thread issues everything, so the loop keeps to counters (no
+                // division): `left` = k-steps left in the current group.
+                uint32_t it = 0, gc = 0, d = tmem_base;
+                int left = 0;
+                bool ok = true;
+                // groups of whole 128-byte stages (every stage: 4 k-steps of one group)
+                const bool aligned = SPG % 4 == 0 && p.K % KG_BK == 0;
+                for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+                    for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                        const int s = it % STAGES;
+                        const uint32_t ph = (it / STAGES) & 1u;
+                        if (!mbar_wait(bar_full(s), ph, abort_flag, p.status, KG_SITE_MMA_FULL)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint64_t da = sdesc_k_sw128(sA + s * KG_A);
+                        const uint64_t db = sdesc_k_sw128(sB + s * KG_B);
+                        const int nk = min(4, KS - 4 * kb);
+                        if (aligned) {
+                            // groups of whole stages: at most one group starts and
+                            // one ends here, so the four MMAs issue back to back
                             if (left == 0) {
-                                // a new group: wait until its slot is drained and re-armed
                                 const uint32_t sl = gc & (KG_NSLOT - 1);
                                 if (!mbar_wait(bar_sempty(sl), (gc / KG_NSLOT) & 1u, abort_flag, p.status,
                                                KG_SITE_MMA_SLOT)) {
+                                    mma_commit(bar_empty(s));
                                     ok = false;
                                     break;
                                 }
@@ -252,26 +268,53 @@ w8a8_kgroup_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                                 d = tmem_base + sl * KG_BN;
                                 left = SPG;
                             }
-                            // +32 bytes along K inside the swizzle atom = +2 in the descriptor
-                            mma_i8(d, da + 2u * k, db + 2u * k, IDESC, 1u);
-                            if (--left == 0) {
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) mma_i8(d, da + 2u * k, db + 2u * k, IDESC, 1u);
+                            left -= 4;
+                            if (left == 0) {
                                 mma_commit(bar_afull(gc & (KG_NSLOT - 1)));
                                 ++gc;
                             }
+                            mma_commit(bar_empty(s));  // stage free once these MMAs finish
+                            continue;
                         }
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            if (k < nk && ok) {
+                                if (left == 0) {
+                                    // a new group: wait until its slot is drained and re-armed
+                                    const uint32_t sl = gc & (KG_NSLOT - 1);
+                                    if (!mbar_wait(bar_sempty(sl), (gc / KG_NSLOT) & 1u, abort_flag, p.status,
+                                                   KG_SITE_MMA_SLOT)) {
+                                        ok = false;
+                                        break;
+                                    }
+                                    tc_fence_after();
+                                    d = tmem_base + sl * KG_BN;
+                                    left = SPG;
+                                }
+                                // +32 bytes along K inside the swizzle atom = +2 in the descriptor
+                                mma_i8(d, da + 2u * k, db + 2u * k, IDESC, 1u);
+                                if (--left == 0) {
+                                    mma_commit(bar_afull(gc & (KG_NSLOT - 1)));
+                                    ++gc;
+                                }
+                            }
+                        }
+                        mma_commit(bar_empty(s));  // stage free once these MMAs finish
+                        if (!ok) break;
                     }
-                    mma_commit(bar_empty(s));  // stage free once these MMAs finish
-                    if (!ok) break;
                 }
+                mma_commit(bar_drain);
+                mbar_wait(bar_drain, 0u, nullptr, p.status, KG_SITE_DRAIN);
             }
-            mma_commit(bar_drain);
-            mbar_wait(bar_drain, 0u, nullptr, p.status, KG_SITE_DRAIN);
-        }
-        __syncwarp();
+            __syncwarp();
+        }  // warps 2-3: idle
     } else {
         // ------------------------------------------------ epilogue
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(KG_REG_HIGH));
         griddep_wait();  // token scales come from the previous grid; y may still be read by it
-        const int ew = warp - 2;
+        const int ew = warp - 4;
         const int quarter = warp & 3;      // TMEM lanes 32*quarter .. +31
         const int col0 = (ew >> 2) * COLS;  // this warp's columns of the tile
         const int r = quarter * 32 + lane;
@@ -326,6 +369,7 @@ w8a8_kgroup_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         for (int i = 0; i < KG_PF; ++i) prefetch();
         uint32_t gc = 0;  // item index
         int slot = 0;     // gc % KG_RING
+        int prev_sl = -1;  // accumulator slot read last, released once its re-arm stores complete
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
             int mt, nt;
             kg_tile(tile, m_tiles, n_tiles, p.group_m, mt, nt);
@@ -338,7 +382,8 @@ w8a8_kgroup_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             for (int g = 0; g < NG; ++g, ++gc) {
                 const uint32_t sl = gc & (KG_NSLOT - 1);
                 const uint32_t par = (gc / KG_NSLOT) & 1u;
-                prefetch();  // item gc + KG_PF
+                __syncwarp();  // every lane is done with the ring slot refilled next
+                prefetch();    // item gc + KG_PF
                 cp_async_wait<KG_PF>();  // this item's scales have landed (own lane) ...
                 const bool got = mbar_wait(bar_afull(sl), par, abort_flag, p.status, KG_SITE_EPI_SLOT);
                 if (!__all_sync(0xFFFFFFFFu, got)) {  // ... and every lane's (warp barrier)
@@ -349,25 +394,32 @@ w8a8_kgroup_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                 const uint32_t ta = tmem_base + lane_off + (uint32_t)(sl * KG_BN + col0);
                 const float4* sc = reinterpret_cast<const float4*>(ring + slot * COLS);
                 slot = slot == KG_RING - 1 ? 0 : slot + 1;
+                // one TMEM round trip for all of this warp's columns
+                uint32_t v[NCH][32];
 #pragma unroll
-                for (int ch = 0; ch < NCH; ++ch) {
-                    uint32_t v[32];
-                    tmem_ld_32x32b_x32(ta + ch * 32, v);
-                    tmem_ld_wait();
-                    tmem_st_splat_x32(ta + ch * 32, kMagicBits);  // re-arm the cells just read
+                for (int ch = 0; ch < NCH; ++ch) tmem_ld_32x32b_x32(ta + ch * 32, v[ch]);
+                tmem_ld_wait();
+                // the previous slot's re-arm stores overlapped this slot's loads:
+                // release it now
+                if (prev_sl >= 0) {
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar_sempty(prev_sl));
+                }
+#pragma unroll
+                for (int ch = 0; ch < NCH; ++ch) tmem_st_splat_x32(ta + ch * 32, kMagicBits);  // re-arm
+                prev_sl = (int)sl;
+#pragma unroll
+                for (int ch = 0; ch < NCH; ++ch)
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         const float4 s4 = sc[ch * 8 + q];  // same address in every lane: a broadcast
-                        const uint64_t a01 = f2_sub(u2_pack(v[4 * q], v[4 * q + 1]), magic2);
-                        const uint64_t a23 = f2_sub(u2_pack(v[4 * q + 2], v[4 * q + 3]), magic2);
+                        const uint64_t a01 = f2_sub(u2_pack(v[ch][4 * q], v[ch][4 * q + 1]), magic2);
+                        const uint64_t a23 = f2_sub(u2_pack(v[ch][4 * q + 2], v[ch][4 * q + 3]), magic2);
                         run[ch * 16 + 2 * q] = f2_fma(f2_pack(s4.x, s4.y), a01, run[ch * 16 + 2 * q]);
                         run[ch * 16 + 2 * q + 1] = f2_fma(f2_pack(s4.z, s4.w), a23, run[ch * 16 + 2 * q + 1]);
                     }
-                }
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar_sempty(sl));
             }
             if (!alive) break;
             // y = act(s_tok * run + bias), one 32x32 box per chunk through a TMA store
@@ -407,6 +459,12 @@ w8a8_kgroup_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                     bulk_commit();
                 }
             }
+        }
+        if (prev_sl >= 0) {  // release the last slot read
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_sempty(prev_sl));
         }
         cp_async_wait<0>();  // no scale copy outstanding at exit
         if (lane == 0) bulk_wait_all();
@@ -464,13 +522,26 @@ int kg_launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& t
         if (rc) return rc;
         attr_set[dev] = true;
     }
+    // setmaxnreg.inc waits until the registers it asks for are free, so the
+    // split must fit the registers the block is launched with
+    static int launch_regs[kMaxDevices] = {};
+    if (!launch_regs[dev]) {
+        cudaFuncAttributes fa;
+        int rc = cuda_status(cudaFuncGetAttributes(&fa, kern));
+        if (rc) return rc;
+        launch_regs[dev] = fa.numRegs;
+    }
+    if ((uint32_t)launch_regs[dev] * KG_THREADS < 128 * KG_REG_LOW + 256 * KG_REG_HIGH) {
+        set_cuda_error(cudaErrorInvalidConfiguration);
+        return ZQ_ERR_CUDA;
+    }
     const int tiles = ((p.M + KG_BM - 1) / KG_BM) * ((p.N + KG_BN - 1) / KG_BN);
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute at[1];
     cfg.attrs = at;
     cfg.numAttrs = (unsigned)pdl_attr(at[0]);
     cfg.gridDim = dim3((unsigned)(tiles < di.sm_count ? tiles : di.sm_count));
-    cfg.blockDim = dim3(64 + 32 * EW);
+    cfg.blockDim = dim3(KG_THREADS);
     cfg.dynamicSmemBytes = kSmem;
     cfg.stream = st;
     count_launch();
