@@ -558,15 +558,16 @@ def kernel_source_hash(sources=PROFILED_SOURCES):
 
 def recorded_traffic(workload, stage):
     """DRAM bytes per launch of the stage's kernel from a committed ncu capture
-    (profiles/dram_traffic.json), if it was taken on the current sources."""
+    (profiles/dram_traffic.json), if it was taken on the current version of
+    the source files the record lists."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
     e = d.get(f"{workload}:{stage}")
-    srcs = KGROUP_SOURCES if workload == "gptj_qkv_kgroups" and stage == "linear1" else PROFILED_SOURCES
-    if not e or e.get("source_hash") != kernel_source_hash(srcs):
+    # the record names the source files its hash covers
+    if not e or e.get("source_hash") != kernel_source_hash(tuple(e.get("sources", PROFILED_SOURCES))):
         return None
     return e.get("dram_bytes")
 
