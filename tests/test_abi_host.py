@@ -123,3 +123,95 @@ def test_max_k_is_the_int32_bound():
 ])
 def test_row_entry_points_reject_bad_arguments_on_host(call, status):
     assert call(zq.lib()) == status
+
+
+Z = zq  # short alias for the status and enum names below
+
+
+@pytest.mark.parametrize("call,status", [
+    # SmoothQuant: calibration and fold
+    (lambda L: L.zq_smooth_calibrate(None, 1, 64, 768, A16, A16, 1e-5, A16, None), Z.ZQ_ERR_NULL),
+    (lambda L: L.zq_smooth_calibrate(A16, 1, 64, 768, A16, A16, 1e-5, None, None), Z.ZQ_ERR_NULL),
+    (lambda L: L.zq_smooth_calibrate(A16, 3, 64, 768, A16, A16, 1e-5, A16, None), Z.ZQ_ERR_DTYPE),
+    (lambda L: L.zq_smooth_calibrate(A16, 1, 64, 760, A16, A16, 1e-5, A16, None), Z.ZQ_ERR_SHAPE),
+    (lambda L: L.zq_smooth_calibrate(A16, 1, 64, 32768 + 16, A16, A16, 1e-5, A16, None), Z.ZQ_ERR_SHAPE),
+    (lambda L: L.zq_smooth_calibrate(MIS, 1, 64, 768, A16, A16, 1e-5, A16, None), Z.ZQ_ERR_ALIGN),
+    (lambda L: L.zq_smooth_weights(None, 64, 768, A16, 0.5, A16, A16, A16b, A16c, A16c, A16b, None),
+     Z.ZQ_ERR_NULL),
+    (lambda L: L.zq_smooth_weights(A16, 64, 768, A16, 0.5, A16, A16, A16b, None, A16c, A16b, None),
+     Z.ZQ_ERR_NULL),                                   # gamma given, gamma_out missing
+    (lambda L: L.zq_smooth_weights(A16, 64, 768, A16, 1.5, A16, A16, A16b, A16c, A16c, A16b, None),
+     Z.ZQ_ERR_DTYPE),                                  # alpha outside [0, 1]
+    (lambda L: L.zq_smooth_weights(A16, 64, 760, A16, 0.5, A16, A16, A16b, A16c, A16c, A16b, None),
+     Z.ZQ_ERR_SHAPE),
+    (lambda L: L.zq_smooth_weights(A16, 64, 768, A16, 0.5, A16, A16, MIS, A16c, A16c, A16b, None),
+     Z.ZQ_ERR_ALIGN),
+    # LLM.int8(): selection, fp16 operands, the linear with the outlier epilogue
+    (lambda L: L.zq_llmint8_select(None, 768, 6.0, A16, A16, A16b, A16c, A16, A16, None), Z.ZQ_ERR_NULL),
+    (lambda L: L.zq_llmint8_select(A16, 760, 6.0, A16, A16, A16b, A16c, A16, A16, None), Z.ZQ_ERR_SHAPE),
+    (lambda L: L.zq_llmint8_select(A16 + 2, 768, 6.0, A16, A16, A16b, A16c, A16, A16, None), Z.ZQ_ERR_ALIGN),
+    (lambda L: L.zq_llmint8_outlier_act(A16, 2, 64, 768, A16, A16, 1e-5, A16b, A16c, A16, None),
+     Z.ZQ_ERR_DTYPE),
+    (lambda L: L.zq_llmint8_outlier_act(A16, 1, 64, 768, A16, A16, 1e-5, A16b, A16c, MIS, None),
+     Z.ZQ_ERR_ALIGN),
+    (lambda L: L.zq_llmint8_outlier_weights(A16, 256, 768, None, A16c, A16, None), Z.ZQ_ERR_NULL),
+    (lambda L: L.zq_llmint8_outlier_weights(A16, 256, 760, A16b, A16c, A16, None), Z.ZQ_ERR_SHAPE),
+    (lambda L: L.zq_w8a8_linear_llmint8(A16, A16b, 64, 128, A16c, A16b, 256, 16, None, 0,
+                                        Z.ZQ_OUT_I8_REQUANT, A16, A16, A16, None), Z.ZQ_ERR_DTYPE),
+    (lambda L: L.zq_w8a8_linear_llmint8(A16, A16b, 64, 128, A16c, A16b, 256, 16, None, 0,
+                                        Z.ZQ_OUT_BF16, None, A16, A16, None), Z.ZQ_ERR_NULL),
+    (lambda L: L.zq_w8a8_linear_llmint8(A16, A16b, 64, 128, A16c, A16b, 256, 48, None, 0,
+                                        Z.ZQ_OUT_BF16, A16, A16, A16, None), Z.ZQ_ERR_SHAPE),
+    (lambda L: L.zq_w8a8_linear_llmint8(A16, A16b, 64, 128, A16c, A16b, 256, 16, None, 0,
+                                        Z.ZQ_OUT_BF16, MIS, A16, A16, None), Z.ZQ_ERR_ALIGN),
+    # the requantizing linear with library-owned scratch
+    (lambda L: L.zq_w8a8_linear_requant_noalloc(A16, A16b, 64, 128, A16c, A16b, 256, 16, None, 0, A16, None,
+                                                None), Z.ZQ_ERR_NULL),
+    (lambda L: L.zq_w8a8_linear_requant_noalloc(A16, A16b, 64, 128, A16c, A16b, 256, 16, None, 2, A16, A16b,
+                                                None), Z.ZQ_ERR_DTYPE),
+    (lambda L: L.zq_w8a8_linear_requant_noalloc(A16, A16b, 64, 120, A16c, A16b, 256, 16, None, 0, A16, A16b,
+                                                None), Z.ZQ_ERR_SHAPE),
+    (lambda L: L.zq_w8a8_linear_requant_noalloc(A16, A16b, 65536, 128, A16c, A16b, 4096, 16, None, 0, A16,
+                                                A16b, None), Z.ZQ_ERR_SCRATCH),   # 1 GiB of fp32 rows
+    # K-axis weight groups: quantizer and linear
+    (lambda L: L.zq_quantize_weights_kgroups(None, 64, 256, 32, A16, A16b, None), Z.ZQ_ERR_NULL),
+    (lambda L: L.zq_quantize_weights_kgroups(A16, 64, 250, 25, A16, A16b, None), Z.ZQ_ERR_SHAPE),  # K % 16
+    (lambda L: L.zq_quantize_weights_kgroups(A16, 64, 256, 48, A16, A16b, None), Z.ZQ_ERR_SHAPE),  # K % G
+    (lambda L: L.zq_quantize_weights_kgroups(A16, 64, 256, 0, A16, A16b, None), Z.ZQ_ERR_SHAPE),
+    (lambda L: L.zq_quantize_weights_kgroups(A16, 64, 256, 32, MIS, A16b, None), Z.ZQ_ERR_ALIGN),
+    (lambda L: L.zq_quantize_weights_kgroups(A16, 64, 256, 32, A16, A16b + 2, None), Z.ZQ_ERR_ALIGN),
+])
+def test_extension_entry_points_reject_bad_arguments_on_host(call, status):
+    assert call(zq.lib()) == status
+
+
+def _kg(**kw):
+    a = dict(xq=A16, s_tok=A16b, T=64, K=256, Wq=A16c, s_w=A16b, N=256, G=128, bias=None, act=0,
+             out=zq.ZQ_OUT_BF16, y=A16, stream=None)
+    a.update(kw)
+    return zq.lib().zq_w8a8_linear_kgroups(a["xq"], a["s_tok"], a["T"], a["K"], a["Wq"], a["s_w"], a["N"],
+                                           a["G"], a["bias"], a["act"], a["out"], a["y"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(xq=None), zq.ZQ_ERR_NULL),
+    (dict(s_tok=None), zq.ZQ_ERR_NULL),
+    (dict(s_w=None), zq.ZQ_ERR_NULL),
+    (dict(y=None), zq.ZQ_ERR_NULL),
+    (dict(out=zq.ZQ_OUT_I8_REQUANT), zq.ZQ_ERR_DTYPE),
+    (dict(out=zq.ZQ_OUT_I32_RAW), zq.ZQ_ERR_DTYPE),
+    (dict(act=2), zq.ZQ_ERR_DTYPE),
+    (dict(T=0), zq.ZQ_ERR_SHAPE),
+    (dict(G=16), zq.ZQ_ERR_SHAPE),             # narrower than one 32-value k-step
+    (dict(G=96), zq.ZQ_ERR_SHAPE),             # K % G
+    (dict(K=512, G=512), zq.ZQ_ERR_SHAPE),     # above 256 columns
+    (dict(N=250), zq.ZQ_ERR_SHAPE),            # N % 16
+    (dict(xq=MIS), zq.ZQ_ERR_ALIGN),
+    (dict(Wq=MIS), zq.ZQ_ERR_ALIGN),
+    (dict(y=MIS), zq.ZQ_ERR_ALIGN),
+    (dict(s_w=A16b + 4), zq.ZQ_ERR_ALIGN),     # scales: 16-byte alignment, as documented
+    (dict(bias=A16 + 4), zq.ZQ_ERR_ALIGN),     # bias too (16-byte loads)
+    (dict(s_tok=A16b + 2), zq.ZQ_ERR_ALIGN),
+])
+def test_kgroup_linear_rejects_bad_arguments_on_host(kw, status):
+    assert _kg(**kw) == status
