@@ -101,6 +101,8 @@ LINEAR_SHAPES = [
     (257, 1024, 384, 256, 1, "bf16"),  # a group spans two stages
     (1000, 4096, 1536, 128, 0, "f32"),  # several waves of tiles, 32 groups
     (513, 2048, 640, 32, 1, "f32"),   # 64 groups, the fp32-sum bound above 1e-5
+    (192, 8192, 256, 64, 0, "f32"),   # 128 groups
+    (64, 12288, 256, 256, 1, "bf16"),  # K = 12288: 48 groups of two stages
 ]
 
 
@@ -126,6 +128,21 @@ def test_linear_kgroups_without_bias_and_repeated_calls(zq):
     zero = np.zeros(N, np.float32)
     ref = oracle.linear_kgroups(xq, st, Wq, sw, G)
     _check(host(y1), ref, _magnitude(xq, st, Wq, sw, G, zero), _tol(K, G, "f32"))
+
+
+def test_linear_kgroups_zero_token_rows_give_the_bias(zq):
+    """Rows whose codes and token scale are all zero (an all-zero input row)
+    come out as exactly the bias; the other rows are unaffected."""
+    T, K, N, G = 160, 512, 272, 128
+    xq, st, Wq, sw, bias = _linear_case(T, K, N, G, 21)
+    zero_rows = [0, 77, 159]
+    xq[zero_rows] = 0
+    st[zero_rows] = 0.0
+    y = host(zq.zq_w8a8_linear_kgroups(dev(xq), dev(st), dev(Wq), dev(np.ascontiguousarray(sw.T)), G,
+                                       bias=dev(bias), out_kind=zq.ZQ_OUT_F32))
+    np.testing.assert_array_equal(y[zero_rows], np.broadcast_to(bias, (len(zero_rows), N)))
+    ref = oracle.linear_kgroups(xq, st, Wq, sw, G, bias)
+    _check(y, ref, _magnitude(xq, st, Wq, sw, G, bias), _tol(K, G, "f32"))
 
 
 def test_gptj_qkv_kgroups_sampled_rows(zq):
