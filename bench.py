@@ -10,6 +10,12 @@ default workload is the BERT-base-shaped FFN block:
       -> W2 [768, 3072] INT8 GEMM + dequant + bias -> bf16 [4096, 768].
 Weight group quantization is offline (done once before timing).
 
+Other workloads (--workload): gptj_qkv (LN + 2048x4096 -> 12288, 128-row
+weight groups), neox_decode (16 tokens, 6144 -> 24576), tiny, gemm_sweep_<M>,
+ln_sweep_<T>_<H>, bert_smooth (SmoothQuant calibration + weight fold),
+bert_llmint8 (LLM.int8() decomposition on BERT W1), gptj_qkv_kgroups (the
+GPT-J projection with 128-column K-axis weight groups).
+
 Metric: INT8 tera-operations per second of the whole step (2*T*N*K integer
 ops per GEMM, summed, over the step time), with the fused LN/token-quant
 bandwidth and the per-kernel roofline alongside.
