@@ -39,6 +39,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -120,11 +121,13 @@ def barrier():
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """nvidia-smi samples (every 200 ms) of the GPU this rank uses."""
+    """nvidia-smi samples (every 200 ms, timestamped) of the GPU this rank
+    uses; stats() summarises the samples of one time window."""
 
-    QUERY = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    QUERY = ("timestamp,index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, uuid: str | None):
         self.uuid = uuid
@@ -145,11 +148,11 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
 
     def stop(self):
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return
         time.sleep(0.25)
         self.proc.terminate()
         try:
@@ -157,21 +160,45 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.thread.join(timeout=5)
+
+    def _rows(self):
+        from datetime import datetime
         rows = []
-        for ln in self.lines:
+        for t_read, ln in list(self.lines):
             f = [x.strip() for x in ln.split(",")]
-            if len(f) < 10:
+            if len(f) < 11:
                 continue
-            if self.uuid and self.uuid not in f[1]:
+            if self.uuid and self.uuid not in f[2]:
                 continue
-            rows.append(f)
+            try:
+                t = datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                t = t_read
+            rows.append((t, f))
+        return rows
+
+    def stats(self, window=None):
+        """Median SM clock under load, max clock and throttle reasons of the
+        samples inside `window` (t0, t1) (all samples when None; the nearest
+        one when the window holds none)."""
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = self._rows()
+        if window is not None and rows:
+            t0, t1 = window
+            inside = [r for r in rows if t0 - 0.1 <= r[0] <= t1 + 0.1]
+            if not inside:
+                mid = 0.5 * (t0 + t1)
+                inside = [min(rows, key=lambda r: abs(r[0] - mid))]
+            rows = inside
+        rows = [f for _, f in rows]
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
-        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i] == "Active"})
-        loaded = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
+        num = lambda v: v.replace(".", "").isdigit()
+        sm = [float(r[3]) for r in rows if num(r[3])]
+        mx = [float(r[4]) for r in rows if num(r[4])]
+        reasons = sorted({self.REASONS[i] for r in rows for i in range(4) if r[7 + i] == "Active"})
+        loaded = [v for v in sm if mx and v > 0.5 * max(mx)] or sm
         return {"sm_mhz": statistics.median(loaded) if loaded else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
 
@@ -195,9 +222,13 @@ class Workload:
         self.config = {}
 
     def dev(self, a):
+        if isinstance(a, self.torch.Tensor):      # drawn on the device already
+            return a
         return self.torch.from_numpy(np.ascontiguousarray(a)).to(self.device)
 
     def dev_act(self, a):
+        if isinstance(a, self.torch.Tensor):
+            return a
         if a.bf16 is not None:
             return self.torch.from_numpy(a.bf16.view(np.int16)).to(self.device).view(self.torch.bfloat16)
         return self.dev(a.f32)
@@ -334,8 +365,36 @@ def build_kgroup_workload(W, zq, torch, device):
     return W
 
 
-def build_workload(name, zq, torch, device):
+def _device_inputs(name, device):
+    """The workload drawn on the GPU (same shapes and distributions as the
+    numpy recipe; used for the large sub-records of the default run)."""
+    from w8a8_post_quantized_b200 import inputs_device as idev
+    if name == "gptj_qkv":
+        return idev.gptj_qkv(device)
+    if name == "gptj_ffn":
+        return idev.gptj_ffn(device)
+    if name == "neox_decode":
+        return idev.neox_decode(device)
+    if name.startswith("gemm_sweep_"):
+        M = int(name.split("_")[-1])
+        return idev.gemm_sweep_point(device, M, inputs.GEMM_SWEEP_M.index(M))
+    if name.startswith("ln_sweep_"):
+        T, H = (int(v) for v in name.split("_")[-2:])
+        idx = inputs.LN_SWEEP_T.index(T) * len(inputs.LN_SWEEP_H) + inputs.LN_SWEEP_H.index(H)
+        return idev.ln_sweep_point(device, T, H, idx)
+    raise SystemExit(f"no device generator for {name}")
+
+
+def _x_dtype(x):
+    if hasattr(x, "dtype") and isinstance(x.dtype, str):
+        return x.dtype
+    return "bf16" if str(x.dtype).endswith("bfloat16") else "f32"
+
+
+def build_workload(name, zq, torch, device, source="host"):
     W = Workload(name, zq, torch, device)
+    if source == "device":
+        return build_linear_workload(W, _device_inputs(name, device), zq, torch, device)
     if name == "gptj_qkv_kgroups":
         return build_kgroup_workload(W, zq, torch, device)
     if name == "bert_smooth":
@@ -353,13 +412,21 @@ def build_workload(name, zq, torch, device):
         T, H = (int(v) for v in name.split("_")[-2:])
         idx = inputs.LN_SWEEP_T.index(T) * len(inputs.LN_SWEEP_H) + inputs.LN_SWEEP_H.index(H)
         w = inputs.ln_sweep_point(T, H, idx)
+    elif name == "gptj_ffn":
+        return build_linear_workload(W, _device_inputs(name, device), zq, torch, device)
     else:
         raise SystemExit(f"unknown workload {name}")
+    return build_linear_workload(W, w, zq, torch, device)
+
+
+def build_linear_workload(W, w, zq, torch, device):
+    """Quantizer (LN + quant, or plain token quant) followed by the workload's
+    linears; every linear but the last requantizes its output per token."""
     x = W.dev_act(w.x)
     T, K = x.shape
     W.tokens = T
     xbytes = x.numel() * x.element_size()
-    W.config = {"workload": w.name, "tokens": T, "hidden": K, "x_dtype": w.x.dtype}
+    W.config = {"workload": w.name, "tokens": T, "hidden": K, "x_dtype": _x_dtype(w.x)}
     q1 = torch.empty((T, K), dtype=torch.int8, device=device)
     st1 = torch.empty(T, dtype=torch.float32, device=device)
     if w.gamma is not None:
@@ -381,6 +448,7 @@ def build_workload(name, zq, torch, device):
     for lin in w.layers:
         Wq, sg = zq.zq_quantize_weights(W.dev(lin.W), lin.group_rows)
         layers.append((Wq, sg, W.dev(lin.bias), lin.group_rows))
+        lin.W = None          # the fp32 weights are not needed once quantized
     torch.cuda.synchronize()
     a_q, a_s = q1, st1
     for i, (Wq, sg, b, G) in enumerate(layers):
@@ -428,27 +496,36 @@ def build_workload(name, zq, torch, device):
 
 # ------------------------------------------------------------------ timing
 
-def time_device(W, steps, warmup, torch):
+def time_device(W, steps, warmup, torch, min_window_s=0.0):
     """Flush L2 before each step; CUDA events on the launching stream.
 
     The step time comes from one CUDA graph holding the whole step (its
     kernels chained by programmatic dependent launch, as a serving loop would
-    replay them).  The per-stage times come from a second timed run in which
-    every stage is its own graph with events between them; they include each
-    stage's own launch latency, so they are upper bounds on the kernels.
-    Returns per-step ms and per-stage ms lists."""
+    replay them), each replay preceded by an L2 flush outside the events.
+
+    The per-stage kernel times come from graphs of [flush; stage] and of
+    [flush] alone, each replayed `steps` times between two events: the
+    stage's time is the difference divided by `steps`.  Both graphs pay the
+    same launch cost, so it cancels, and every stage launch starts on a cold
+    L2, as in the step.  With min_window_s > 0 the number of timed steps
+    grows until the step timing spans at least that long (so clock samples
+    fall inside it).  Returns (per-step ms list, {stage: ms}, steps timed)."""
     stream = torch.cuda.current_stream()
     flush = L2Flush(torch, W.device)
     for _, fn in W.stages:       # eager warm-up (sets kernel attributes, loads modules)
         fn()
     torch.cuda.synchronize()
-    graphs = []
     cap = torch.cuda.Stream()
     cap.wait_stream(stream)
     with torch.cuda.stream(cap):
+        flush_g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(flush_g, stream=cap):
+            flush()
+        graphs = []
         for label, fn in W.stages:
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=cap):
+                flush()
                 fn()
             graphs.append((label, g))
         whole = torch.cuda.CUDAGraph()
@@ -457,7 +534,6 @@ def time_device(W, steps, warmup, torch):
                 fn()
     stream.wait_stream(cap)
     torch.cuda.synchronize()
-    n = len(graphs)
 
     def run_step(k):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(k)]
@@ -468,31 +544,35 @@ def time_device(W, steps, warmup, torch):
             evs[s][1].record(stream)
         return evs
 
-    def run_stages(k):
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(k)]
-        for s in range(k):
-            flush()
-            evs[s][0].record(stream)
-            for i, (_, g) in enumerate(graphs):
-                g.replay()
-                evs[s][i + 1].record(stream)
-        return evs
+    def replay_ms(g, k):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(k):
+            g.replay()
+        b.record(stream)
+        b.synchronize()
+        return a.elapsed_time(b)
 
-    run_step(warmup)
+    evs = run_step(warmup)
     torch.cuda.synchronize()
+    if min_window_s > 0:
+        est = statistics.median(a.elapsed_time(b) for a, b in evs) + replay_ms(flush_g, 3) / 3
+        steps = max(steps, min(4000, int(math.ceil(min_window_s * 1e3 / max(est, 1e-3)))))
     barrier()
     torch.cuda.synchronize()
     evs = run_step(steps)
     torch.cuda.synchronize()
     barrier()
     per_step = [a.elapsed_time(b) for a, b in evs]
-    run_stages(warmup)
-    torch.cuda.synchronize()
-    evs = run_stages(steps)
-    torch.cuda.synchronize()
-    per_stage = {label: [e[i].elapsed_time(e[i + 1]) for e in evs] for i, (label, _) in enumerate(graphs)}
-    del graphs, whole
-    return per_step, per_stage
+    k = max(steps, 20)
+    for _, g in graphs:
+        replay_ms(g, 2)
+    stage_ms = {}
+    for label, g in graphs:
+        diffs = [(replay_ms(g, k) - replay_ms(flush_g, k)) / k for _ in range(3)]
+        stage_ms[label] = max(statistics.median(diffs), 1e-4)
+    del graphs, whole, flush_g
+    return per_step, stage_ms, steps
 
 
 def time_e2e(W, steps, warmup, torch):
@@ -701,6 +781,71 @@ def oracle_kgroup_sample(budget_s=12.0, max_rows=None):
 
 # -------------------------------------------------------------------- main
 
+# Sub-records of the default run: the other workloads, each timed on its own
+# after the headline (inputs drawn on the device).  GEMM sweep M = 16 / 256
+# are HBM-bound (weight stream), M = 4096 / 16384 tensor-bound; the LN sweep
+# points are those of at least 32 MB of input.
+SUBRECORDS = ("gptj_qkv", "gptj_ffn", "neox_decode", "gemm_sweep_16", "gemm_sweep_256", "gemm_sweep_4096",
+              "gemm_sweep_16384", "ln_sweep_16384_1024", "ln_sweep_16384_4096", "ln_sweep_16384_12288",
+              "ln_sweep_65536_1024", "ln_sweep_65536_4096", "ln_sweep_65536_12288")
+
+
+def stage_roofline(W, label, ms, peaks, workload):
+    """Achieved rate of one stage's kernel(s) against the roofline that binds it."""
+    bound, units, _ = W.kernel_units[label]
+    int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+    if bound == "tensor":
+        achieved = units / (ms * 1e-3) / 1e12
+        return {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(int8_peak, 1), "unit": "TOPS",
+                "frac": round(achieved / int8_peak, 4),
+                "peak_source": f"{peaks['source']} bf16 burst x {INT8_OVER_BF16:g} (nominal int8/bf16)",
+                "frac_vs_spec": round(achieved / SPEC_INT8_TOPS, 4),
+                "traffic": recorded_traffic(workload, label), "kernel_ms": round(ms, 5)}
+    achieved = units / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(achieved / peaks["hbm_gbs"], 4), "peak_source": f"{peaks['source']} copy bandwidth",
+            "frac_vs_spec": round(achieved / SPEC_HBM_GBS, 4),
+            "traffic": recorded_traffic(workload, label), "kernel_ms": round(ms, 5)}
+
+
+def step_value(W, ms_per_step, world=1):
+    """(metric, unit, value) of the whole step: INT8 TOPS when the step has
+    GEMMs, else GB/s of algorithmic bytes."""
+    if W.ops:
+        return ("W8A8 linear INT8 TOPS (whole step, incl. fused LN/token-quant)", "TOPS",
+                world * W.ops / (ms_per_step * 1e-3) / 1e12)
+    qb = sum(v[1] for v in W.kernel_units.values() if v[0] == "hbm")
+    return (W.metric or "fused LN/token-quant GB/s", "GB/s", world * (W.bytes or qb) / (ms_per_step * 1e-3) / 1e9)
+
+
+def dominant_stage(stage_ms, stage_launches):
+    """The longest stage that is a single launch of one kernel."""
+    single = [k for k in stage_ms if stage_launches.get(k) == 1]
+    return max(single or list(stage_ms), key=lambda k: stage_ms[k])
+
+
+def measure_subrecord(name, zq, torch, device, steps, warmup, peaks, clocks):
+    W = build_workload(name, zq, torch, device, source="device")
+    launches, stage_launches = count_launches(W, zq, torch)
+    t0 = time.time()
+    per_step, stage_ms, n = time_device(W, steps, warmup, torch, min_window_s=0.3)
+    t1 = time.time()
+    zq.zq_device_status()
+    ms = statistics.mean(per_step)
+    metric, unit, value = step_value(W, ms)
+    dom = dominant_stage(stage_ms, stage_launches)
+    rec = {"value": round(value, 2), "unit": unit, "ms_per_step": round(ms, 5), "steps": n,
+           "tokens_per_s": round(W.tokens / (ms * 1e-3), 1),
+           "config": dict(W.config, inputs="drawn on the device (torch CUDA generator), numpy recipe's distributions"),
+           "stages_ms": {k: round(v, 5) for k, v in stage_ms.items()},
+           "stage_roofline": {k: stage_roofline(W, k, v, peaks, name) for k, v in stage_ms.items()},
+           "dominant": dom, "gpu_launches": launches * n, "clocks": clocks.stats((t0, t1))}
+    rec["roofline"] = dict(rec["stage_roofline"][dom], kernel=dom)
+    del W
+    torch.cuda.empty_cache()
+    return rec
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -710,6 +855,9 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-subrecords", action="store_true",
+                    help="time only the selected workload (default run: also the other workloads)")
+    ap.add_argument("--subrecords", default=None, help="comma-separated sub-record workloads to time")
     a = ap.parse_args(argv)
     if a.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -735,8 +883,9 @@ def main(argv=None):
     props = torch.cuda.get_device_properties(device)
     clocks = ClockSampler(str(getattr(props, "uuid", "")) or None)
     clocks.start()
-    per_step, per_stage = time_device(W, a.steps, a.warmup, torch)
-    clk = clocks.stop()
+    t0 = time.time()
+    per_step, stage_ms, _ = time_device(W, a.steps, a.warmup, torch)
+    t1 = time.time()
     zq.zq_device_status()
     local_ms = sum(per_step)
     max_ms = reduce_max(local_ms)
@@ -747,40 +896,15 @@ def main(argv=None):
     zq.zq_device_status()
 
     peaks = load_peaks()
-    int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
-    stage_ms = {k: statistics.mean(v) for k, v in per_stage.items()}
-    # dominant kernel: the longest stage that is a single launch of one kernel
-    single = [k for k in stage_ms if stage_launches.get(k) == 1]
-    dom = max(single or list(stage_ms), key=lambda k: stage_ms[k])
-    bound, units, kind = W.kernel_units[dom]
-    if bound == "tensor":
-        achieved = units / (stage_ms[dom] * 1e-3) / 1e12
-        roof = {"kernel": f"w8a8 linear ({dom})", "bound": "tensor", "achieved": round(achieved, 1),
-                "peak": round(int8_peak, 1), "unit": "TOPS", "frac": round(achieved / int8_peak, 4),
-                "peak_source": f"{peaks['source']} bf16 burst x {INT8_OVER_BF16:g} (nominal int8/bf16)",
-                "frac_vs_spec": round(achieved / SPEC_INT8_TOPS, 4),
-                "traffic": recorded_traffic(a.workload, dom), "stage_ms": round(stage_ms[dom], 5)}
-    else:
-        achieved = units / (stage_ms[dom] * 1e-3) / 1e9
-        roof = {"kernel": dom if dom.endswith("quant") else f"w8a8 linear ({dom})", "bound": "hbm",
-                "achieved": round(achieved, 1),
-                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "peak_source": f"{peaks['source']} copy bandwidth",
-                "frac_vs_spec": round(achieved / SPEC_HBM_GBS, 4),
-                "traffic": recorded_traffic(a.workload, dom), "stage_ms": round(stage_ms[dom], 5)}
+    dom = dominant_stage(stage_ms, stage_launches)
+    roof = dict(stage_roofline(W, dom, stage_ms[dom], peaks, a.workload),
+                kernel=dom if dom.endswith("quant") else f"w8a8 linear ({dom})")
     qlabel = "ln_quant" if "ln_quant" in stage_ms else ("act_quant" if "act_quant" in stage_ms else None)
     qb = W.kernel_units[qlabel][1] if qlabel else 0
     q_gbs = qb / (stage_ms[qlabel] * 1e-3) / 1e9 if qlabel else None
 
-    if W.ops:
-        metric, unit = "W8A8 linear INT8 TOPS (whole step, incl. fused LN/token-quant)", "TOPS"
-        value = world * W.ops / (ms_per_step * 1e-3) / 1e12
-        e2e_value = world * W.ops / (e2e_ms * 1e-3) / 1e12
-    else:
-        metric, unit = W.metric or "fused LN/token-quant GB/s", "GB/s"
-        step_bytes = W.bytes or qb
-        value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
-        e2e_value = world * step_bytes / (e2e_ms * 1e-3) / 1e9
+    metric, unit, value = step_value(W, ms_per_step, world)
+    e2e_value = value * ms_per_step / e2e_ms
 
     out = {
         "metric": metric, "value": round(value, 2), "unit": unit, "n_gpus": world,
@@ -790,9 +914,12 @@ def main(argv=None):
         "data": "synthetic (seeded; layer shapes only, random weights)",
         "config": dict(W.config, parallelism=f"replicas x{world}",
                        l2="flushed before every timed step (256 MiB write + read-back)",
-                       timing="one CUDA graph per step (kernels chained by programmatic dependent launch), CUDA events on the launching stream; per-stage times from per-stage graphs"),
+                       timing="one CUDA graph per step (kernels chained by programmatic dependent launch), "
+                              "CUDA events on the launching stream; per-stage kernel times from graphs of "
+                              "[flush; stage] minus graphs of [flush], replayed back to back"),
         "tokens_per_s": round(world * W.tokens / (ms_per_step * 1e-3), 1),
         "stages_ms": {k: round(v, 5) for k, v in stage_ms.items()},
+        "stage_roofline": {k: stage_roofline(W, k, v, peaks, a.workload) for k, v in stage_ms.items()},
         "ln_quant_gbs": round(q_gbs, 1) if q_gbs else None,
         "ln_quant_frac_hbm": round(q_gbs / peaks["hbm_gbs"], 4) if q_gbs else None,
         "roofline": roof,
@@ -800,13 +927,26 @@ def main(argv=None):
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": launches_per_step * a.steps,
         "launches_per_stage": stage_launches,
-        "clocks": clk,
+        "clocks": clocks.stats((t0, t1)),
     }
-    if rank == 0 and world == 1 and not a.no_cpu_baseline and W.ops:
+    has_ops = bool(W.ops)
+    del W
+    torch.cuda.empty_cache()
+    # the other workloads, one GPU only (replica runs time the headline alone)
+    names = SUBRECORDS if a.subrecords is None else tuple(n for n in a.subrecords.split(",") if n)
+    if world == 1 and a.workload == "bert_ffn" and not a.no_subrecords and names:
+        subs = {}
+        for name in names:
+            subs[name] = measure_subrecord(name, zq, torch, device, max(10, min(a.steps, 20)), a.warmup, peaks,
+                                           clocks)
+        out["subrecords"] = subs
+        out["clocks_all"] = clocks.stats()
+    clocks.stop()
+    if rank == 0 and world == 1 and not a.no_cpu_baseline and has_ops:
         ops, secs, rows, T = oracle_sample(a.workload, budget_s=a.cpu_budget)
         out["cpu_baseline"] = {"value": round(ops / secs / 1e12, 8), "unit": unit, "cores": 1,
                                "kind": "oracle",
-                               "sample": f"{rows} of {T} token rows of {W.config['workload']}, "
+                               "sample": f"{rows} of {T} token rows of {out['config']['workload']}, "
                                          f"plain C oracle, single thread, {secs:.1f} s"}
     if rank == 0:
         print(json.dumps(out), flush=True)

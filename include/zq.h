@@ -181,9 +181,12 @@ int zq_linear_block(const void* x, int x_dtype, int64_t T, int64_t K,
 
 /* ---- requantizing linear without caller scratch ---------------------------
  * No counterpart on the source pages: this entry point exists for callers,
- * not for the method.  It computes exactly what zq_w8a8_linear computes with
- * out_kind = ZQ_OUT_I8_REQUANT (same kernels, same results), but takes no
- * workspace and allocates nothing.
+ * not for the method.  It computes what zq_w8a8_linear computes with
+ * out_kind = ZQ_OUT_I8_REQUANT, but takes no workspace and allocates nothing.
+ * It always takes the scratch route (GEMM with an fp32 epilogue output and a
+ * per-token absmax, then a requantization kernel), while zq_w8a8_linear may
+ * take a fused kernel for the same shape; the two then agree within one code
+ * on at most 0.1% of the codes, and their scales within 1e-5 relative.
  *
  * Who needs it: callers that cannot obtain device memory themselves -- code
  * running inside a host framework that owns every device allocation and
@@ -196,8 +199,10 @@ int zq_linear_block(const void* x, int x_dtype, int64_t T, int64_t K,
  * exits.  A call needs round_up(4*T, 256) + 4*T*N bytes of it; a larger
  * problem returns ZQ_ERR_SCRATCH before anything is enqueued.
  * Set-up: the first call on each device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current); make that first call
- * before any stream capture.
+ * (cudaGetSymbolAddress, with that device current) and keeps it for the life
+ * of the process; make that first call before any stream capture.  Do not
+ * call this entry point on a device after cudaDeviceReset of that device:
+ * the module is then loaded again and the kept address may be stale.
  * Sharing: all calls on a device use the same array and it keeps the last
  * call's contents (the call clears what must start at zero).  Calls whose
  * GPU work overlaps -- on different streams, or from different threads --

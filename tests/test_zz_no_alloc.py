@@ -3,9 +3,10 @@
 memory themselves -- e.g. plugins of a host framework that owns every device
 allocation, or serving loops where cudaMalloc is not allowed after start-up.
 
-The GPU test calls it through the C ABI twice in a row (the library's fixed
-scratch array keeps the first call's contents when the second starts) and
-compares each result with the workspace-taking entry point,
+The GPU test calls it through the C ABI on several problems in a row (the
+library's fixed scratch array keeps the previous call's contents when the
+next starts) and compares each result with the CPU oracle's requantizing
+linear and with the workspace-taking entry point,
 zq_w8a8_linear(..., ZQ_OUT_I8_REQUANT), within the tolerances the other
 tests use.  This file is collected last so that a run stopping at the first
 failure has already run every other test; it also passes on its own in a
@@ -16,17 +17,19 @@ import numpy as np
 import pytest
 import torch
 
-from tests.gpu_helpers import assert_codes_close, assert_scales_close, host
+import oracle
+from tests.gpu_helpers import assert_codes_close, assert_scales_close, dev, host, sample_rows
 from w8a8_post_quantized_b200 import zq
 
 
-def _inputs(T, K, N, G, seed):
-    g = torch.Generator(device="cuda").manual_seed(seed)
-    xq = torch.randint(-127, 128, (T, K), dtype=torch.int8, device="cuda", generator=g)
-    Wq = torch.randint(-127, 128, (N, K), dtype=torch.int8, device="cuda", generator=g)
-    s_tok = torch.rand(T, device="cuda", generator=g) * 0.05 + 1e-3
-    s_grp = torch.rand(N // G, device="cuda", generator=g) * 1e-3 + 1e-5
-    bias = torch.randn(N, device="cuda", generator=g) * 0.01
+def _case(T, K, N, G, seed):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_t(4.0, size=(T, K)).astype(np.float32)
+    x[:, rng.permutation(K)[: max(1, K // 100)]] *= 25.0
+    W = (0.02 * rng.standard_normal((N, K))).astype(np.float32)
+    bias = (0.01 * rng.standard_normal(N)).astype(np.float32)
+    xq, s_tok = oracle.quantize_rows(x)
+    Wq, s_grp = oracle.quantize_weights(W, G)
     return xq, s_tok, Wq, s_grp, bias
 
 
@@ -41,23 +44,32 @@ def _call_noalloc(xq, s_tok, Wq, s_grp, G, bias, y, s_out):
 
 
 @pytest.mark.gpu
-def test_noalloc_requant_matches_workspace_entry_point_twice():
-    cases = [(4096, 768, 3072, 64, 11),     # the BERT W1 layer: 48 MiB of the 64 MiB array
-             (300, 512, 400, 80, 12)]       # smaller, ragged, run second over stale contents
-    outs = []
-    for T, K, N, G, seed in cases:
-        xq, s_tok, Wq, s_grp, bias = _inputs(T, K, N, G, seed)
+def test_noalloc_requant_matches_oracle_and_workspace_entry_point():
+    # (T, K, N, G, seed, rows checked against the oracle: None = all)
+    cases = [(4096, 768, 3072, 64, 11, 96),    # the BERT W1 layer: 48 MiB of the 64 MiB array
+             (300, 512, 400, 80, 12, None),    # small and ragged, over the first call's contents
+             (300, 256, 5120, 128, 13, None),  # an output row wider than 4096 features
+             (300, 512, 400, 80, 14, None)]    # the second shape again, new data
+    for T, K, N, G, seed, n_rows in cases:
+        xq, s_tok, Wq, s_grp, bias = _case(T, K, N, G, seed)
+        d = [dev(a) for a in (xq, s_tok, Wq, s_grp, bias)]
         y = torch.empty((T, N), dtype=torch.int8, device="cuda")
         s_out = torch.empty(T, dtype=torch.float32, device="cuda")
-        assert _call_noalloc(xq, s_tok, Wq, s_grp, G, bias, y, s_out) == zq.ZQ_OK
+        assert _call_noalloc(d[0], d[1], d[2], d[3], G, d[4], y, s_out) == zq.ZQ_OK
         zq.zq_device_status()
-        ref_y, ref_s = zq.zq_w8a8_linear(xq, s_tok, Wq, s_grp, G, bias=bias, act=zq.ZQ_ACT_GELU,
+        qh, sh = host(y), host(s_out)
+        # against the oracle (all rows, or the last block and a seeded sample)
+        rows = (np.arange(T) if n_rows is None else
+                np.unique(np.concatenate([np.arange(T - 128, T), sample_rows(T, n_rows, seed=seed)])))
+        q_ref, s_ref = oracle.linear_requant(xq[rows], s_tok[rows], Wq, s_grp, G, bias, oracle.ACT_GELU)
+        assert_codes_close(qh[rows], q_ref)
+        assert_scales_close(sh[rows], s_ref)
+        # against the workspace-taking entry point (every row)
+        ref_y, ref_s = zq.zq_w8a8_linear(d[0], d[1], d[2], d[3], G, bias=d[4], act=zq.ZQ_ACT_GELU,
                                          out_kind=zq.ZQ_OUT_I8_REQUANT)
         zq.zq_device_status()
-        assert_codes_close(host(y), host(ref_y))
-        assert_scales_close(host(s_out), host(ref_s))
-        outs.append(host(s_out))
-    assert outs[0].shape != outs[1].shape
+        assert_codes_close(qh, host(ref_y))
+        assert_scales_close(sh, host(ref_s))
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():

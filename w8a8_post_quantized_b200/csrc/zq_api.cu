@@ -22,6 +22,11 @@ static std::atomic<uint64_t> g_launches{0};
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
+std::mutex& launch_cache_mutex() {
+    static std::mutex mu;
+    return mu;
+}
+
 int pdl_attr(cudaLaunchAttribute& attr) {
     static const bool off = getenv("ZQ_NO_PDL") != nullptr;
     if (off) return 0;

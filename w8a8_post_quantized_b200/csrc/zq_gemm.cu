@@ -604,6 +604,7 @@ template <typename K>
 int max_clusters(K kern, int S, size_t smem, int threads, int dev) {
     static int cache[kMaxDevices][9] = {};
     if (S < 1 || S > 8) return 0;
+    std::lock_guard<std::mutex> lk(launch_cache_mutex());
     if (cache[dev][S] == 0) {
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute at[1];
@@ -637,11 +638,14 @@ int launch_cfg(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& 
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= kMaxDevices) return ZQ_ERR_DEVICE;
-    if (!attr_set[dev]) {
-        int rc = cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                  (int)kSmem));
-        if (rc) return rc;
-        attr_set[dev] = true;
+    {
+        std::lock_guard<std::mutex> lk(launch_cache_mutex());
+        if (!attr_set[dev]) {
+            int rc = cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                      (int)kSmem));
+            if (rc) return rc;
+            attr_set[dev] = true;
+        }
     }
     const int tiles = ((p.M + BM - 1) / BM) * ((p.N + BN - 1) / BN);
     if constexpr (SWAP) {
@@ -740,16 +744,20 @@ int pick_bn(int64_t T, int64_t N, int sms) {
 
 }  // namespace
 
+static PFN_cuTensorMapEncodeTiled_v12000 lookup_encode_fn() {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    return nullptr;
+}
+
+// looked up once per process (a function-local static is initialised once,
+// even when several threads make their first call together)
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
-                                             &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = lookup_encode_fn();
     return fn;
 }
 

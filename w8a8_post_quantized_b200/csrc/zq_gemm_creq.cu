@@ -389,6 +389,7 @@ int launch_w8a8_requant_cluster(const LinearArgs& a, const DeviceInfo& di, cudaS
     static bool attr_set[kMaxDevices] = {};
     static int max_clusters[kMaxDevices][kMaxCluster + 1] = {};
     int rc;
+    std::unique_lock<std::mutex> lk(launch_cache_mutex());
     if (!attr_set[dev]) {
         if ((rc = cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))))
             return rc;
@@ -415,9 +416,11 @@ int launch_w8a8_requant_cluster(const LinearArgs& a, const DeviceInfo& di, cudaS
             max_clusters[dev][C] = n;
         }
     }
-    if (max_clusters[dev][C] < 1) return ZQ_ERR_SHAPE;
+    const int max_ncl = max_clusters[dev][C];
+    lk.unlock();
+    if (max_ncl < 1) return ZQ_ERR_SHAPE;
     const int64_t m_tiles = (a.T + BM - 1) / BM;
-    const int ncl = (int)(m_tiles < max_clusters[dev][C] ? m_tiles : max_clusters[dev][C]);
+    const int ncl = (int)(m_tiles < max_ncl ? m_tiles : max_ncl);
     cfg.gridDim = dim3(ncl * C);
     cfg.numAttrs = 1 + (unsigned)pdl_attr(attr[1]);
 

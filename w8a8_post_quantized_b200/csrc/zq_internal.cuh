@@ -9,6 +9,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "zq.h"
 
 namespace zq {
@@ -648,6 +650,10 @@ void count_launch();  // every kernel launch goes through this
 // before touching global memory.
 int pdl_attr(cudaLaunchAttribute& attr);
 int cuda_status(cudaError_t e);  // ZQ_OK or ZQ_ERR_CUDA (and records the text)
+// Guards the launchers' per-device caches (kernel attributes set, occupancy
+// and register counts queried once per device), which several host threads
+// may fill at the same time on their first calls.
+std::mutex& launch_cache_mutex();
 
 // launchers (no validation; the C ABI validates)
 int launch_quantize_weights(const float* W, int64_t N, int64_t K, int64_t G, int8_t* Wq,

@@ -517,6 +517,7 @@ int kg_launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& t
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= kMaxDevices) return ZQ_ERR_DEVICE;
+    std::unique_lock<std::mutex> lk(launch_cache_mutex());
     if (!attr_set[dev]) {
         int rc = cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem));
         if (rc) return rc;
@@ -531,7 +532,9 @@ int kg_launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& t
         if (rc) return rc;
         launch_regs[dev] = fa.numRegs;
     }
-    if ((uint32_t)launch_regs[dev] * KG_THREADS < 128 * KG_REG_LOW + 256 * KG_REG_HIGH) {
+    const int regs = launch_regs[dev];
+    lk.unlock();
+    if ((uint32_t)regs * KG_THREADS < 128 * KG_REG_LOW + 256 * KG_REG_HIGH) {
         set_cuda_error(cudaErrorInvalidConfiguration);
         return ZQ_ERR_CUDA;
     }

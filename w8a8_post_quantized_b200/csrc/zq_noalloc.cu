@@ -16,7 +16,9 @@
 // library holds ZQ_NOALLOC_SCRATCH_BYTES of device memory for it until the
 // process exits.  Host code cannot use its name as a device address, so the
 // first call on each device looks the address up with cudaGetSymbolAddress
-// (with that device current) and caches it.
+// (with that device current) and caches it for the life of the process, so
+// the entry point must not be used on a device after cudaDeviceReset of it
+// (the module, and with it the array, may then be loaded at a new address).
 #include <mutex>
 
 #include "zq_internal.cuh"
