@@ -55,6 +55,7 @@ WIDE_SHAPES = [
     (16, 768, 6144, 64),      # decode-sized: swapped operand roles, 16 tokens
     (33, 1024, 4096, 64),     # swapped, 33 tokens
     (64, 512, 8192, 128),     # swapped, 64 tokens, wide
+    (130, 64, 38144, 16),     # 149 column tiles per row: more than the SMs, the scratch route
 ]
 
 

@@ -27,6 +27,18 @@ std::mutex& launch_cache_mutex() {
     return mu;
 }
 
+int requant_route() {
+    static const int route = [] {
+        const char* v = getenv("ZQ_REQUANT_ROUTE");
+        if (!v) return 0;
+        if (!strcmp(v, "cluster")) return 1;
+        if (!strcmp(v, "grid")) return 2;
+        if (!strcmp(v, "scratch")) return 3;
+        return 0;
+    }();
+    return route;
+}
+
 int pdl_attr(cudaLaunchAttribute& attr) {
     static const bool off = getenv("ZQ_NO_PDL") != nullptr;
     if (off) return 0;
@@ -149,9 +161,17 @@ int run_linear(const int8_t* xq, const float* s_tok, int64_t T, int64_t K, const
     a.s_tok_out = s_tok_out;
     int rc;
     if (out_kind == ZQ_OUT_I8_REQUANT) {
-        // fused: the row absmax is exchanged inside a thread-block cluster
-        rc = launch_w8a8_requant_cluster(a, di, st);
-        if (rc != ZQ_ERR_SHAPE) return rc;
+        const int route = requant_route();
+        // fused: the row absmax is exchanged inside a thread-block cluster (N <= 4096)
+        if (route == 0 || route == 1) {
+            rc = launch_w8a8_requant_cluster(a, di, st);
+            if (rc != ZQ_ERR_SHAPE) return rc;
+        }
+        // fused, any width: the row absmax is exchanged through global memory
+        if (route == 0 || route == 2) {
+            rc = launch_w8a8_requant_grid(a, static_cast<uint32_t*>(ws), di, st);
+            if (rc != ZQ_ERR_SHAPE) return rc;
+        }
         // otherwise: fp32 epilogue output + row absmax in the workspace, then requantize
         uint8_t* w = static_cast<uint8_t*>(ws);
         a.h_ws = reinterpret_cast<float*>(w);

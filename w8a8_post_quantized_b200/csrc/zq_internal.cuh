@@ -704,6 +704,17 @@ int launch_w8a8_gemm_outliers(const LinearArgs& a, const uint16_t* xo, const uin
 // a thread-block cluster (no scratch).  ZQ_ERR_SHAPE: shape not covered (the
 // caller then uses the scratch path).
 int launch_w8a8_requant_cluster(const LinearArgs& a, const DeviceInfo& di, cudaStream_t st);
+// Requantizing linear for rows of any width in one persistent kernel: the
+// per-token absmax goes through global atomics and per-row-block arrival
+// counters in `scratch` (requant_grid_scratch_bytes(T) bytes, zeroed by the
+// launcher).  ZQ_ERR_SHAPE: shape not covered (T <= 64, or more column tiles
+// per row than co-resident CTAs).
+size_t requant_grid_scratch_bytes(int64_t T);
+int launch_w8a8_requant_grid(const LinearArgs& a, uint32_t* scratch, const DeviceInfo& di, cudaStream_t st);
+// Which requantizing route zq_w8a8_linear takes: 0 = automatic, 1 = cluster
+// kernel only, 2 = grid kernel only, 3 = scratch route (environment variable
+// ZQ_REQUANT_ROUTE = cluster | grid | scratch; for measurements).
+int requant_route();
 // int8 matrix [rows, K] as a TMA tensor: box 128 bytes of K x box_rows rows,
 // 128-byte swizzle, out-of-range elements read as 0.
 int make_tmap_i8(CUtensorMap* tm, const void* ptr, int64_t rows, int64_t K, int box_rows);
