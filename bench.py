@@ -858,6 +858,8 @@ def main(argv=None):
     ap.add_argument("--no-subrecords", action="store_true",
                     help="time only the selected workload (default run: also the other workloads)")
     ap.add_argument("--subrecords", default=None, help="comma-separated sub-record workloads to time")
+    ap.add_argument("--inputs", default="host", choices=["host", "device"],
+                    help="draw the selected workload's inputs with numpy (host) or on the GPU (device)")
     a = ap.parse_args(argv)
     if a.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -876,7 +878,7 @@ def main(argv=None):
     from w8a8_post_quantized_b200 import zq
     zq.lib()
 
-    W = build_workload(a.workload, zq, torch, device)
+    W = build_workload(a.workload, zq, torch, device, source=a.inputs)
     launches_per_step, stage_launches = count_launches(W, zq, torch)
     zq.zq_device_status()
 

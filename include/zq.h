@@ -155,7 +155,12 @@ int zq_act_quant(const void* x, int x_dtype, int64_t T, int64_t H,
  * bias == NULL.
  * workspace : device scratch of at least zq_w8a8_linear_workspace(...)
  *          bytes (may be NULL when that is 0).  Its contents on entry do not
- *          matter; it is clobbered.
+ *          matter; it is clobbered.  Only ZQ_OUT_I8_REQUANT needs one: with
+ *          T > 64 and at most one column tile of 256 per SM of the current
+ *          device a word per token and per 128-token block (the fused
+ *          kernels), else the fp32 output plus a word per token.  The query
+ *          reads the current device's SM count; with no usable device it
+ *          returns the larger size.
  * Constraints: K % 16 == 0, N % 16 == 0, N % G == 0, K <= ZQ_MAX_K.
  * Errors: NULL, SHAPE, ALIGN, OVERFLOW, DTYPE, WORKSPACE, CUDA, DEVICE. */
 size_t zq_w8a8_linear_workspace(int64_t T, int64_t K, int64_t N, int out_kind);
@@ -182,11 +187,8 @@ int zq_linear_block(const void* x, int x_dtype, int64_t T, int64_t K,
 /* ---- requantizing linear without caller scratch ---------------------------
  * No counterpart on the source pages: this entry point exists for callers,
  * not for the method.  It computes what zq_w8a8_linear computes with
- * out_kind = ZQ_OUT_I8_REQUANT, but takes no workspace and allocates nothing.
- * It always takes the scratch route (GEMM with an fp32 epilogue output and a
- * per-token absmax, then a requantization kernel), while zq_w8a8_linear may
- * take a fused kernel for the same shape; the two then agree within one code
- * on at most 0.1% of the codes, and their scales within 1e-5 relative.
+ * out_kind = ZQ_OUT_I8_REQUANT, through the same kernels and with the same
+ * results, but takes no workspace and allocates nothing.
  *
  * Who needs it: callers that cannot obtain device memory themselves -- code
  * running inside a host framework that owns every device allocation and
@@ -196,15 +198,21 @@ int zq_linear_block(const void* x, int x_dtype, int64_t T, int64_t K,
  *
  * Scratch: one array of ZQ_NOALLOC_SCRATCH_BYTES in device memory, owned by
  * the library.  Every GPU that loads the library holds it until the process
- * exits.  A call needs round_up(4*T, 256) + 4*T*N bytes of it; a larger
- * problem returns ZQ_ERR_SCRATCH before anything is enqueued.
+ * exits.  What a call needs of it depends on the kernel the shape takes:
+ * nothing for T > 64 and N <= 4096 (the row absmax is exchanged inside a
+ * thread-block cluster); 4 * (T + ceil(T / 128)) bytes, rounded up to 256,
+ * for T > 64 and wider rows (per-token absmax words and per-row-block
+ * counters); round_up(4*T*N, 256) + round_up(4*T, 256) bytes otherwise (at
+ * most 64 tokens, or rows of more column tiles of 256 than the GPU has SMs:
+ * the fp32 output and the absmax words).  A call that needs more than the
+ * array returns ZQ_ERR_SCRATCH before anything is enqueued.
  * Set-up: the first call on each device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current) and keeps it for the life
  * of the process; make that first call before any stream capture.  Do not
  * call this entry point on a device after cudaDeviceReset of that device:
  * the module is then loaded again and the kept address may be stale.
  * Sharing: all calls on a device use the same array and it keeps the last
- * call's contents (the call clears what must start at zero).  Calls whose
+ * call's contents (each call clears what must start at zero).  Calls whose
  * GPU work overlaps -- on different streams, or from different threads --
  * race on the array and give wrong results; order them on one stream.
  * Arguments, layouts and the other errors as zq_w8a8_linear: y is int8

@@ -50,8 +50,18 @@ def test_status_strings_and_version():
         assert txt and txt.decode()
     assert L.zq_status_string(12345).decode() == "unknown status"
     assert zq.zq_version() >= 100
-    assert zq.lib().zq_w8a8_linear_workspace(4096, 768, 3072, zq.ZQ_OUT_I8_REQUANT) >= 4096 * 3072 * 4
     assert zq.lib().zq_w8a8_linear_workspace(4096, 768, 3072, zq.ZQ_OUT_BF16) == 0
+    # at most 64 tokens: the fp32 output and the absmax words
+    assert zq.lib().zq_w8a8_linear_workspace(64, 768, 3072, zq.ZQ_OUT_I8_REQUANT) >= 64 * 3072 * 4 + 64 * 4
+
+
+def test_requant_workspace_without_a_device():
+    """With no usable device the query cannot tell whether the fused kernels
+    apply and asks for the scratch route's size (fp32 output + absmax words)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    assert zq.lib().zq_w8a8_linear_workspace(4096, 768, 3072, zq.ZQ_OUT_I8_REQUANT) >= 4096 * 3072 * 4 + 4096 * 4
 
 
 def _lin(**kw):
@@ -171,8 +181,8 @@ Z = zq  # short alias for the status and enum names below
                                                 None), Z.ZQ_ERR_DTYPE),
     (lambda L: L.zq_w8a8_linear_requant_noalloc(A16, A16b, 64, 120, A16c, A16b, 256, 16, None, 0, A16, A16b,
                                                 None), Z.ZQ_ERR_SHAPE),
-    (lambda L: L.zq_w8a8_linear_requant_noalloc(A16, A16b, 65536, 128, A16c, A16b, 4096, 16, None, 0, A16,
-                                                A16b, None), Z.ZQ_ERR_SCRATCH),   # 1 GiB of fp32 rows
+    (lambda L: L.zq_w8a8_linear_requant_noalloc(A16, A16b, 64, 128, A16c, A16b, 300000, 16, None, 0, A16,
+                                                A16b, None), Z.ZQ_ERR_SCRATCH),   # 77 MB of fp32 rows
     # K-axis weight groups: quantizer and linear
     (lambda L: L.zq_quantize_weights_kgroups(None, 64, 256, 32, A16, A16b, None), Z.ZQ_ERR_NULL),
     (lambda L: L.zq_quantize_weights_kgroups(A16, 64, 250, 25, A16, A16b, None), Z.ZQ_ERR_SHAPE),  # K % 16

@@ -13,6 +13,7 @@ seeded sample of the others (each oracle row depends only on that row of
 the inputs)."""
 import numpy as np
 import pytest
+import torch
 
 import oracle
 from tests.gpu_helpers import assert_codes_close, assert_scales_close, dev, host, sample_rows
@@ -89,3 +90,23 @@ def test_requant_gptj_ffn_up_sampled_rows(zq):
     assert_codes_close(qh[rows], q_ref)
     assert_scales_close(sh[rows], s_ref)
     assert np.all(np.abs(qh).max(axis=1) == 127)
+
+
+def test_requant_workspace_is_small_when_fused(zq):
+    """More than 64 tokens and at most one column tile per SM: the fused
+    kernels need a word per row and per 128-row block, not the fp32 output;
+    a call given exactly that workspace runs, a smaller one is refused."""
+    T, K, N, G = 300, 256, 5120, 128
+    need = zq.lib().zq_w8a8_linear_workspace(T, K, N, zq.ZQ_OUT_I8_REQUANT)
+    assert 4 * (T + 3) <= need < 4 * T * N
+    xq, s_tok, Wq, s_grp, bias = _case(T, K, N, G, seed=99)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    q, s = zq.zq_w8a8_linear(dev(xq), dev(s_tok), dev(Wq), dev(s_grp), G, bias=dev(bias), act=zq.ZQ_ACT_GELU,
+                             out_kind=zq.ZQ_OUT_I8_REQUANT, workspace=ws)
+    q_ref, s_ref = oracle.linear_requant(xq, s_tok, Wq, s_grp, G, bias, oracle.ACT_GELU)
+    assert_codes_close(host(q), q_ref)
+    assert_scales_close(host(s), s_ref)
+    with pytest.raises(zq.ZQError) as e:
+        zq.zq_w8a8_linear(dev(xq), dev(s_tok), dev(Wq), dev(s_grp), G, bias=dev(bias), act=zq.ZQ_ACT_GELU,
+                          out_kind=zq.ZQ_OUT_I8_REQUANT, workspace=ws[: need - 256])
+    assert e.value.status == zq.ZQ_ERR_WORKSPACE

@@ -3,13 +3,17 @@
 memory themselves -- e.g. plugins of a host framework that owns every device
 allocation, or serving loops where cudaMalloc is not allowed after start-up.
 
-The GPU test calls it through the C ABI on several problems in a row (the
-library's fixed scratch array keeps the previous call's contents when the
-next starts) and compares each result with the CPU oracle's requantizing
-linear and with the workspace-taking entry point,
-zq_w8a8_linear(..., ZQ_OUT_I8_REQUANT), within the tolerances the other
-tests use.  This file is collected last so that a run stopping at the first
-failure has already run every other test; it also passes on its own in a
+It takes the same kernels as the workspace-taking entry point
+zq_w8a8_linear(..., ZQ_OUT_I8_REQUANT), with the library's fixed scratch
+array in place of the workspace: per-token absmax words and row-block
+counters for rows wider than 4096 features, the fp32 output for at most 64
+tokens, nothing at all for the cluster kernel.  The GPU test calls it
+through the C ABI on several problems in a row, each route twice (the array
+keeps the previous call's contents when the next starts), and compares each
+result with the CPU oracle's requantizing linear and with the
+workspace-taking entry point, within the tolerances the other tests use.
+This file is collected last so that a run stopping at the first failure
+has already run every other test; it also passes on its own in a
 fresh process (the first call does the per-device set-up)."""
 import ctypes
 
@@ -46,10 +50,12 @@ def _call_noalloc(xq, s_tok, Wq, s_grp, G, bias, y, s_out):
 @pytest.mark.gpu
 def test_noalloc_requant_matches_oracle_and_workspace_entry_point():
     # (T, K, N, G, seed, rows checked against the oracle: None = all)
-    cases = [(4096, 768, 3072, 64, 11, 96),    # the BERT W1 layer: 48 MiB of the 64 MiB array
-             (300, 512, 400, 80, 12, None),    # small and ragged, over the first call's contents
-             (300, 256, 5120, 128, 13, None),  # an output row wider than 4096 features
-             (300, 512, 400, 80, 14, None)]    # the second shape again, new data
+    cases = [(300, 256, 5120, 128, 13, None),  # rows wider than 4096: absmax words + counters
+             (48, 512, 2048, 64, 15, None),    # 48 tokens: the fp32 output in the array
+             (4096, 768, 3072, 64, 11, 96),    # the BERT W1 layer: the cluster kernel, no scratch
+             (300, 256, 5120, 128, 14, None),  # wide rows again, over the fp32 route's contents
+             (48, 512, 2048, 64, 16, None),    # 48 tokens again, new data
+             (2048, 1024, 16384, 128, 17, 32)] # GPT-J FFN-up width, 2048 tokens
     for T, K, N, G, seed, n_rows in cases:
         xq, s_tok, Wq, s_grp, bias = _case(T, K, N, G, seed)
         d = [dev(a) for a in (xq, s_tok, Wq, s_grp, bias)]
@@ -75,8 +81,11 @@ def test_noalloc_requant_matches_oracle_and_workspace_entry_point():
 def test_noalloc_rejects_problems_beyond_its_scratch():
     """Host-side check, before anything is enqueued (fake pointers are never used)."""
     A = 0x7F0000000000
-    T, N = 4096, 4096                        # 64 MiB of fp32 output alone: does not fit
-    rc = zq.lib().zq_w8a8_linear_requant_noalloc(A, A, T, 768, A, A, N, 64, None, 1, A, A, None)
+    T, N = 64, 300000                        # 64 tokens: 76.8 MB of fp32 output, does not fit
+    rc = zq.lib().zq_w8a8_linear_requant_noalloc(A, A, T, 768, A, A, N, 16, None, 1, A, A, None)
+    assert rc == zq.ZQ_ERR_SCRATCH
+    T, N = 20 << 20, 8192                    # wide rows: 80 MiB of absmax words alone
+    rc = zq.lib().zq_w8a8_linear_requant_noalloc(A, A, T, 64, A, A, N, 64, None, 1, A, A, None)
     assert rc == zq.ZQ_ERR_SCRATCH
     assert zq.ZQ_NOALLOC_SCRATCH_BYTES == 64 << 20
     assert zq.lib().zq_w8a8_linear_requant_noalloc(None, A, 4, 64, A, A, 16, 16, None, 1, A, A,

@@ -114,8 +114,12 @@ inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 size_t linear_ws_bytes(int64_t T, int64_t K, int64_t N, int out_kind) {
     (void)K;
     if (out_kind != ZQ_OUT_I8_REQUANT || T <= 0 || N <= 0) return 0;
-    // fp32 [T, N] epilogue output + [T] absmax words
-    return round_up((size_t)T * (size_t)N * sizeof(float), kWsAlign) + round_up((size_t)T * 4, kWsAlign);
+    // the SM count decides whether the fused kernels cover the shape; without
+    // a usable device assume the scratch route
+    int sms = 0;
+    DeviceInfo di;
+    if (device_info(&di) == ZQ_OK) sms = di.sm_count;
+    return requant_ws_bytes(T, N, sms);
 }
 
 int check_linear(const int8_t* xq, const float* s_tok, int64_t T, int64_t K, const int8_t* Wq,
@@ -144,7 +148,7 @@ int check_linear(const int8_t* xq, const float* s_tok, int64_t T, int64_t K, con
 
 int run_linear(const int8_t* xq, const float* s_tok, int64_t T, int64_t K, const int8_t* Wq,
                const float* s_grp, int64_t N, int64_t G, const float* bias, int act, int out_kind,
-               void* y, float* s_tok_out, void* ws, const DeviceInfo& di, cudaStream_t st) {
+               void* y, float* s_tok_out, void* ws, size_t ws_bytes, const DeviceInfo& di, cudaStream_t st) {
     LinearArgs a{};
     a.xq = xq;
     a.s_tok = s_tok;
@@ -159,31 +163,55 @@ int run_linear(const int8_t* xq, const float* s_tok, int64_t T, int64_t K, const
     a.out_kind = out_kind;
     a.y = y;
     a.s_tok_out = s_tok_out;
-    int rc;
-    if (out_kind == ZQ_OUT_I8_REQUANT) {
-        const int route = requant_route();
-        // fused: the row absmax is exchanged inside a thread-block cluster (N <= 4096)
-        if (route == 0 || route == 1) {
-            rc = launch_w8a8_requant_cluster(a, di, st);
-            if (rc != ZQ_ERR_SHAPE) return rc;
-        }
-        // fused, any width: the row absmax is exchanged through global memory
-        if (route == 0 || route == 2) {
-            rc = launch_w8a8_requant_grid(a, static_cast<uint32_t*>(ws), di, st);
-            if (rc != ZQ_ERR_SHAPE) return rc;
-        }
-        // otherwise: fp32 epilogue output + row absmax in the workspace, then requantize
-        uint8_t* w = static_cast<uint8_t*>(ws);
-        a.h_ws = reinterpret_cast<float*>(w);
-        a.amax_ws = reinterpret_cast<uint32_t*>(w + round_up((size_t)T * N * sizeof(float), kWsAlign));
-        if ((rc = cuda_status(cudaMemsetAsync(a.amax_ws, 0, (size_t)T * 4, st)))) return rc;
-        if ((rc = launch_w8a8_gemm(a, di, st))) return rc;
-        return launch_requant_rows(a.h_ws, T, N, a.amax_ws, static_cast<int8_t*>(y), s_tok_out, di, st);
-    }
+    if (out_kind == ZQ_OUT_I8_REQUANT) return run_requant(a, ws, ws_bytes, ZQ_ERR_WORKSPACE, di, st);
     return launch_w8a8_gemm(a, di, st);
 }
 
 }  // namespace
+
+namespace zq {
+
+size_t requant_scratch_route_bytes(int64_t T, int64_t N) {
+    // fp32 [T, N] epilogue output + [T] absmax words
+    return round_up((size_t)T * (size_t)N * sizeof(float), kWsAlign) + round_up((size_t)T * 4, kWsAlign);
+}
+
+size_t requant_ws_bytes(int64_t T, int64_t N, int sms) {
+    const int64_t n_t = (N + 255) / 256;
+    const int route = requant_route();
+    // T > 64 with at most one column tile per SM: the fused kernels (the
+    // cluster kernel needs none, the grid kernel a word per row and per row block)
+    if (route != 3 && T > 64 && sms > 0 && n_t <= sms) return round_up(requant_grid_scratch_bytes(T), kWsAlign);
+    return requant_scratch_route_bytes(T, N);
+}
+
+int run_requant(const LinearArgs& a0, void* ws, size_t ws_bytes, int err_small, const DeviceInfo& di,
+                cudaStream_t st) {
+    LinearArgs a = a0;
+    const int route = requant_route();
+    int rc;
+    // fused: the row absmax is exchanged inside a thread-block cluster (N <= 4096)
+    if (route == 0 || route == 1) {
+        rc = launch_w8a8_requant_cluster(a, di, st);
+        if (rc != ZQ_ERR_SHAPE) return rc;
+    }
+    // fused, any width: the row absmax is exchanged through global memory
+    if (route == 0 || route == 2) {
+        rc = launch_w8a8_requant_grid(a, static_cast<uint32_t*>(ws), ws_bytes, di, st);
+        if (rc == ZQ_ERR_WORKSPACE) return err_small;
+        if (rc != ZQ_ERR_SHAPE) return rc;
+    }
+    // otherwise: fp32 epilogue output + row absmax in the scratch, then requantize
+    if (!ws || ws_bytes < requant_scratch_route_bytes(a.T, a.N)) return err_small;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    a.h_ws = reinterpret_cast<float*>(w);
+    a.amax_ws = reinterpret_cast<uint32_t*>(w + round_up((size_t)a.T * a.N * sizeof(float), kWsAlign));
+    if ((rc = cuda_status(cudaMemsetAsync(a.amax_ws, 0, (size_t)a.T * 4, st)))) return rc;
+    if ((rc = launch_w8a8_gemm(a, di, st))) return rc;
+    return launch_requant_rows(a.h_ws, a.T, a.N, a.amax_ws, static_cast<int8_t*>(a.y), a.s_tok_out, di, st);
+}
+
+}  // namespace zq
 
 extern "C" {
 
@@ -398,7 +426,7 @@ int zq_w8a8_linear(const int8_t* xq, const float* s_tok, int64_t T, int64_t K, c
     DeviceInfo di;
     if ((rc = device_info(&di))) return rc;
     return run_linear(xq, s_tok, T, K, Wq, s_grp, N, group_rows, bias, act, out_kind, y, s_tok_out,
-                      workspace, di, as_stream(stream));
+                      workspace, workspace_bytes, di, as_stream(stream));
 }
 
 size_t zq_linear_block_workspace(int64_t T, int64_t K, int64_t N, int out_kind) {
@@ -436,7 +464,7 @@ int zq_linear_block(const void* x, int x_dtype, int64_t T, int64_t K, const floa
     else rc = launch_act_quant(x, x_dtype, T, K, nullptr, ZQ_ACT_NONE, xq, s_tok, di, st);
     if (rc) return rc;
     return run_linear(xq, s_tok, T, K, Wq, s_grp, N, group_rows, bias, act, out_kind, y, s_tok_out,
-                      lin_ws, di, st);
+                      lin_ws, lin_bytes, di, st);
 }
 
 }  // extern "C"

@@ -358,10 +358,12 @@ w8a8_requant_grid_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
 }
 
 // Zeroes the absmax words and row-block counters of the requantizing linear.
-// Waits for the previous grid first (an earlier call may still read them).
+// It lets the linear launch at once (its prologue and first weight loads then
+// overlap this kernel and the one before it) but waits for the previous grid
+// before writing (an earlier call may still read the words).
 __global__ void zero_words_kernel(uint32_t* __restrict__ w, int n) {
-    griddep_wait();
     griddep_launch_dependents();
+    griddep_wait();
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) w[i] = 0u;
 }
 
@@ -374,7 +376,8 @@ size_t requant_grid_scratch_bytes(int64_t T) {
     return (size_t)(T + m_tiles) * sizeof(uint32_t);
 }
 
-int launch_w8a8_requant_grid(const LinearArgs& a, uint32_t* scratch, const DeviceInfo& di, cudaStream_t st) {
+int launch_w8a8_requant_grid(const LinearArgs& a, uint32_t* scratch, size_t scratch_bytes, const DeviceInfo& di,
+                             cudaStream_t st) {
     static_assert(smem_bytes() <= 232448, "shared memory budget");
     static_assert(smem_bytes() > 116 * 1024, "one CTA per SM (it owns all of TMEM)");
     const int64_t n_t = (a.N + BN - 1) / BN;
@@ -403,6 +406,7 @@ int launch_w8a8_requant_grid(const LinearArgs& a, uint32_t* scratch, const Devic
         // the CTAs wait on one another: all of them must be resident at once
         if (per_sm[dev] < 1) return ZQ_ERR_SHAPE;
     }
+    if (!scratch || scratch_bytes < requant_grid_scratch_bytes(a.T)) return ZQ_ERR_WORKSPACE;
     uint32_t* amax = scratch;
     uint32_t* count = scratch + a.T;
     const int nwords = (int)(a.T + m_tiles);

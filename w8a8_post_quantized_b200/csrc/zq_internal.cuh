@@ -709,8 +709,21 @@ int launch_w8a8_requant_cluster(const LinearArgs& a, const DeviceInfo& di, cudaS
 // counters in `scratch` (requant_grid_scratch_bytes(T) bytes, zeroed by the
 // launcher).  ZQ_ERR_SHAPE: shape not covered (T <= 64, or more column tiles
 // per row than co-resident CTAs).
+// ZQ_ERR_WORKSPACE: the kernel applies but scratch_bytes is too small
+// (checked before anything is launched).
 size_t requant_grid_scratch_bytes(int64_t T);
-int launch_w8a8_requant_grid(const LinearArgs& a, uint32_t* scratch, const DeviceInfo& di, cudaStream_t st);
+int launch_w8a8_requant_grid(const LinearArgs& a, uint32_t* scratch, size_t scratch_bytes, const DeviceInfo& di,
+                             cudaStream_t st);
+// Scratch of the requantizing linear: the bytes the route for this shape
+// needs on a device with `sms` SMs (sms <= 0: unknown, assume the scratch
+// route), and the bytes of the scratch route (fp32 output + absmax words).
+size_t requant_ws_bytes(int64_t T, int64_t N, int sms);
+size_t requant_scratch_route_bytes(int64_t T, int64_t N);
+// The requantizing linear through its routes (cluster kernel, grid kernel,
+// scratch route) with `ws` as scratch; returns err_small, having launched
+// nothing, when the route the shape takes needs more than ws_bytes.
+int run_requant(const LinearArgs& a, void* ws, size_t ws_bytes, int err_small, const DeviceInfo& di,
+                cudaStream_t st);
 // Which requantizing route zq_w8a8_linear takes: 0 = automatic, 1 = cluster
 // kernel only, 2 = grid kernel only, 3 = scratch route (environment variable
 // ZQ_REQUANT_ROUTE = cluster | grid | scratch; for measurements).

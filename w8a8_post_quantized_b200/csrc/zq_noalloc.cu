@@ -2,10 +2,11 @@
 // caller-supplied scratch memory and allocates none.
 //
 // The requantizing linear (zq_w8a8_linear with ZQ_OUT_I8_REQUANT) needs
-// scratch: the fp32 epilogue output of the whole row block and a per-token
-// absmax word, because the new per-token scale depends on every output
-// feature of the token.  Normally the caller passes that scratch as the
-// workspace.  Some callers cannot obtain device memory on their own: code
+// scratch for most shapes, because the new per-token scale depends on every
+// output feature of the token: per-token absmax words and per-row-block
+// arrival counters (rows wider than 4096 features), or the fp32 epilogue
+// output and the absmax words (at most 64 tokens).  Normally the caller
+// passes that scratch as the workspace.  Some callers cannot obtain device memory on their own: code
 // that runs inside a host framework which owns every device allocation and
 // hands its plugins no workspace, and latency-critical serving loops where a
 // cudaMalloc (which may synchronize the device) is not allowed after start-up.
@@ -48,7 +49,6 @@ int scratch_address(unsigned char** out) {
     return ZQ_OK;
 }
 
-inline size_t round256(size_t v) { return (v + 255) / 256 * 256; }
 inline bool aligned(const void* p, uintptr_t a) { return reinterpret_cast<uintptr_t>(p) % a == 0; }
 
 }  // namespace
@@ -69,17 +69,18 @@ extern "C" int zq_w8a8_linear_requant_noalloc(const int8_t* xq, const float* s_t
     if (!aligned(xq, 16) || !aligned(Wq, 16) || !aligned(y, 16) || !aligned(s_tok, 4) ||
         !aligned(s_grp, 4) || !aligned(s_tok_out, 4) || (bias && !aligned(bias, 4)))
         return ZQ_ERR_ALIGN;
-    // scratch layout: [absmax words, T x 4 bytes][fp32 epilogue output, T x N x 4 bytes]
-    const size_t amax_bytes = round256((size_t)T * 4);
-    const size_t h_bytes = (size_t)T * (size_t)N * sizeof(float);
-    if (amax_bytes + h_bytes > (size_t)ZQ_NOALLOC_SCRATCH_BYTES) return ZQ_ERR_SCRATCH;
+    // The least scratch any route could need for this shape: none for at most
+    // 4096 features (the cluster kernel), a word per row and per row block for
+    // wider rows (the grid kernel), the fp32 output for at most 64 tokens (the
+    // scratch route).  Larger than the array: refused before any device call.
+    const size_t least = T <= 64 ? requant_scratch_route_bytes(T, N) : N <= 4096 ? 0 : requant_grid_scratch_bytes(T);
+    if (least > (size_t)ZQ_NOALLOC_SCRATCH_BYTES) return ZQ_ERR_SCRATCH;
 
     DeviceInfo di;
     int rc = device_info(&di);
     if (rc) return rc;
     unsigned char* scratch = nullptr;
     if ((rc = scratch_address(&scratch))) return rc;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
 
     LinearArgs a{};
     a.xq = xq;
@@ -94,10 +95,10 @@ extern "C" int zq_w8a8_linear_requant_noalloc(const int8_t* xq, const float* s_t
     a.act = act;
     a.out_kind = ZQ_OUT_I8_REQUANT;
     a.y = y;
-    a.amax_ws = reinterpret_cast<uint32_t*>(scratch);
-    a.h_ws = reinterpret_cast<float*>(scratch + amax_bytes);
-    // the array keeps the previous call's contents: the absmax words must start at 0
-    if ((rc = cuda_status(cudaMemsetAsync(a.amax_ws, 0, (size_t)T * 4, st)))) return rc;
-    if ((rc = launch_w8a8_gemm(a, di, st))) return rc;
-    return launch_requant_rows(a.h_ws, T, N, a.amax_ws, y, s_tok_out, di, st);
+    a.s_tok_out = s_tok_out;
+    // the same routes as zq_w8a8_linear, with the array as their scratch; each
+    // route clears what must start at zero (the array keeps the previous
+    // call's contents)
+    return run_requant(a, scratch, (size_t)ZQ_NOALLOC_SCRATCH_BYTES, ZQ_ERR_SCRATCH, di,
+                       static_cast<cudaStream_t>(stream));
 }
