@@ -625,7 +625,7 @@ def count_launches(W, zq, torch):
 # The sources of the hot-path kernels the ncu records describe (the
 # quantizers, both GEMMs, their shared helpers and their launch code).
 PROFILED_SOURCES = ("zq_internal.cuh", "zq_api.cu", "zq_rowquant.cu", "zq_quant.cu", "zq_gemm.cu",
-                    "zq_gemm_creq.cu")
+                    "zq_gemm_creq.cu", "zq_gemm_greq.cu")
 # ... and of the K-axis group linear (its kernel, helpers, tensor-map code)
 KGROUP_SOURCES = ("zq_internal.cuh", "zq_kgroup.cu", "zq_gemm.cu")
 
