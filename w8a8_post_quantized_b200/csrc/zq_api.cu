@@ -181,7 +181,8 @@ size_t requant_ws_bytes(int64_t T, int64_t N, int sms) {
     const int route = requant_route();
     // T > 64 with at most one column tile per SM: the fused kernels (the
     // cluster kernel needs none, the grid kernel a word per row and per row block)
-    if (route != 3 && T > 64 && sms > 0 && n_t <= sms) return round_up(requant_grid_scratch_bytes(T), kWsAlign);
+    if ((route == 0 || route == 2) && T > 64 && sms > 0 && n_t <= sms)
+        return round_up(requant_grid_scratch_bytes(T), kWsAlign);
     return requant_scratch_route_bytes(T, N);
 }
 
