@@ -153,14 +153,23 @@ int zq_act_quant(const void* x, int x_dtype, int64_t T, int64_t H,
  * y[t, o] = act(s_tok[t] * s_grp[o / G] * acc[t, o] + bias[o]) in fp32.
  * ZQ_OUT_I32_RAW stores acc itself and requires act == ZQ_ACT_NONE and
  * bias == NULL.
- * workspace : device scratch of at least zq_w8a8_linear_workspace(...)
- *          bytes (may be NULL when that is 0).  Its contents on entry do not
- *          matter; it is clobbered.  Only ZQ_OUT_I8_REQUANT needs one: with
- *          T > 64 and at most one column tile of 256 per SM of the current
- *          device a word per token and per 128-token block (the fused
- *          kernels), else the fp32 output plus a word per token.  The query
- *          reads the current device's SM count; with no usable device it
- *          returns the larger size.
+ * workspace : device scratch of zq_w8a8_linear_workspace(...) bytes (may
+ *          be NULL when that is 0), 16-byte aligned when not NULL.  Its
+ *          contents on entry do not matter; it is clobbered.
+ *          ZQ_OUT_I8_REQUANT requires it: with T > 64 and at most one column
+ *          tile of 256 per SM of the current device a word per token and per
+ *          128-token block (the fused kernels), else the fp32 output plus a
+ *          word per token.  For the other kinds it is optional: with
+ *          T <= 64 and at least as many 128-row weight tiles as SMs, the
+ *          query returns the size of the int32 partial sums (a 128 x 64
+ *          block and a flag per SM) that let every SM take an equal share
+ *          of the (weight tile, k-block) iterations; given fewer bytes the
+ *          call splits K over thread-block clusters instead, with the same
+ *          results.  The environment variable ZQ_EVEN_SPLIT = off | on
+ *          (read on every call) turns that choice off, or on for every
+ *          T <= 64.  The query reads the current device's SM count; with
+ *          no usable device it returns the requantizing kinds' larger size
+ *          and 0 for the others.
  * Constraints: K % 16 == 0, N % 16 == 0, N % G == 0, K <= ZQ_MAX_K.
  * Errors: NULL, SHAPE, ALIGN, OVERFLOW, DTYPE, WORKSPACE, CUDA, DEVICE. */
 size_t zq_w8a8_linear_workspace(int64_t T, int64_t K, int64_t N, int out_kind);

@@ -39,6 +39,17 @@ int requant_route() {
     return route;
 }
 
+int even_split_mode() {
+    // read on every call (a workspace query and the call it sizes may then
+    // disagree; the workspace is optional where this applies, so a call
+    // whose workspace is too small takes the other route)
+    const char* v = getenv("ZQ_EVEN_SPLIT");
+    if (!v) return 0;
+    if (!strcmp(v, "off")) return 1;
+    if (!strcmp(v, "on")) return 2;
+    return 0;
+}
+
 int pdl_attr(cudaLaunchAttribute& attr) {
     static const bool off = getenv("ZQ_NO_PDL") != nullptr;
     if (off) return 0;
@@ -112,13 +123,14 @@ constexpr size_t kWsAlign = 256;
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 size_t linear_ws_bytes(int64_t T, int64_t K, int64_t N, int out_kind) {
-    (void)K;
-    if (out_kind != ZQ_OUT_I8_REQUANT || T <= 0 || N <= 0) return 0;
-    // the SM count decides whether the fused kernels cover the shape; without
-    // a usable device assume the scratch route
+    if (T <= 0 || N <= 0) return 0;
+    // the SM count decides which kernels cover the shape; without a usable
+    // device assume the scratch route (and no even split)
     int sms = 0;
     DeviceInfo di;
     if (device_info(&di) == ZQ_OK) sms = di.sm_count;
+    if (out_kind != ZQ_OUT_I8_REQUANT)  // optional: the partial sums of the few-token even split
+        return decode_even_applies(T, K, N, sms) ? round_up(decode_sk_ws_bytes(sms), kWsAlign) : 0;
     return requant_ws_bytes(T, N, sms);
 }
 
@@ -138,10 +150,12 @@ int check_linear(const int8_t* xq, const float* s_tok, int64_t T, int64_t K, con
     if (check_x && (!aligned(xq, 16) || !aligned(s_tok, 4))) return ZQ_ERR_ALIGN;
     if (!aligned(Wq, 16) || !aligned(y, 16) || !aligned(s_grp, 4)) return ZQ_ERR_ALIGN;
     if ((bias && !aligned(bias, 4)) || (s_tok_out && !aligned(s_tok_out, 4))) return ZQ_ERR_ALIGN;
-    const size_t need = linear_ws_bytes(T, K, N, out_kind);
-    if (need) {
-        if (!ws || ws_bytes < need) return ZQ_ERR_WORKSPACE;
-        if (!aligned(ws, 16)) return ZQ_ERR_ALIGN;
+    if (ws && !aligned(ws, 16)) return ZQ_ERR_ALIGN;
+    // required for the requantizing kinds; optional otherwise (the few-token
+    // kernels then split K over clusters instead of evenly over all SMs)
+    if (out_kind == ZQ_OUT_I8_REQUANT) {
+        const size_t need = linear_ws_bytes(T, K, N, out_kind);
+        if (need && (!ws || ws_bytes < need)) return ZQ_ERR_WORKSPACE;
     }
     return ZQ_OK;
 }
@@ -164,6 +178,11 @@ int run_linear(const int8_t* xq, const float* s_tok, int64_t T, int64_t K, const
     a.y = y;
     a.s_tok_out = s_tok_out;
     if (out_kind == ZQ_OUT_I8_REQUANT) return run_requant(a, ws, ws_bytes, ZQ_ERR_WORKSPACE, di, st);
+    // few tokens: the even split where it is taken and the workspace holds its partials
+    if (decode_even_applies(T, K, N, di.sm_count) && ws && ws_bytes >= decode_sk_ws_bytes(di.sm_count)) {
+        const int rc = launch_w8a8_decode_sk(a, ws, ws_bytes, di, st);
+        if (rc != ZQ_ERR_SHAPE) return rc;
+    }
     return launch_w8a8_gemm(a, di, st);
 }
 

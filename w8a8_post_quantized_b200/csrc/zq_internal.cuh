@@ -700,6 +700,22 @@ struct LinearArgs {
 int launch_w8a8_gemm(const LinearArgs& a, const DeviceInfo& di, cudaStream_t st);
 int launch_w8a8_gemm_outliers(const LinearArgs& a, const uint16_t* xo, const uint16_t* wo, const DeviceInfo& di,
                               cudaStream_t st);
+// Few-token linear (T <= 64; f32, bf16 or raw int32 output; weights on the
+// MMA's M side) with the (weight tile, k-block) iterations in equal
+// contiguous ranges, one persistent CTA per SM.  A tile that a range boundary
+// cuts is summed from int32 partials in `ws` (decode_sk_ws_bytes(sm_count)
+// bytes, 16-byte aligned), with one ready flag per CTA zeroed by a small
+// kernel launched first.  ZQ_ERR_SHAPE: not covered; ZQ_ERR_WORKSPACE: ws
+// missing or too small (nothing launched); the caller then takes
+// launch_w8a8_gemm.  decode_even_applies: whether the shape takes this route
+// on a device with `sms` SMs (ZQ_EVEN_SPLIT overrides the choice).
+size_t decode_sk_ws_bytes(int sms);
+bool decode_even_applies(int64_t T, int64_t K, int64_t N, int sms);
+int launch_w8a8_decode_sk(const LinearArgs& a, void* ws, size_t ws_bytes, const DeviceInfo& di, cudaStream_t st);
+// 0 = the choice above, 1 = never split evenly, 2 = always when the kernel
+// covers the shape (environment variable ZQ_EVEN_SPLIT = off | on, read on
+// every call; for measurements and tests).
+int even_split_mode();
 // Requantizing linear with the per-token absmax exchanged between the CTAs of
 // a thread-block cluster (no scratch).  ZQ_ERR_SHAPE: shape not covered (the
 // caller then uses the scratch path).
