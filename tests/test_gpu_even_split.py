@@ -148,9 +148,9 @@ def test_repeated_calls_reuse_the_workspace(zq, monkeypatch, T, K, N):
 
 def test_neox_decode_layer_sampled(zq, monkeypatch):
     """The decode layer at full size (16 tokens, 6144 -> 24576, G = 256,
-    GeLU), on the route the cost model picks: bf16 outputs of 512 sampled
-    columns against the oracle on their weight rows; the whole int32 product
-    against the split-K clusters."""
+    GeLU), on the default route (the even split: 192 weight tiles): bf16
+    outputs of 512 sampled columns against the oracle on their weight rows;
+    the whole int32 product against the split-K clusters."""
     monkeypatch.delenv("ZQ_EVEN_SPLIT", raising=False)
     T, K, N, G = 16, 6144, 24576, 256
     rng = np.random.default_rng(2024)
