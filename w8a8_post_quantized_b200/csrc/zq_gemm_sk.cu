@@ -71,7 +71,7 @@ struct SkParams {
     const float* bias;  // may be null
     void* y;            // [Nt, M]
     int act;
-    int32_t* part;      // [gridDim][BM][kMaxBN] partial accumulators
+    int32_t* part;      // [gridDim][kMaxBN columns][BM rows] partial accumulators
     uint32_t* flag;     // [gridDim], zero on entry
     int* status;
 };
@@ -397,9 +397,6 @@ __global__ void zero_flags_kernel(uint32_t* __restrict__ w, int n) {
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) w[i] = 0u;
 }
 
-}  // namespace
-
-namespace {
 int launch_zero_flags(uint32_t* flag, int n, cudaStream_t st) {
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute at[1];
@@ -411,6 +408,7 @@ int launch_zero_flags(uint32_t* flag, int n, cudaStream_t st) {
     count_launch();
     return cuda_status(cudaLaunchKernelEx(&cfg, zero_flags_kernel, flag, n));
 }
+
 }  // namespace
 
 bool decode_even_applies(int64_t T, int64_t K, int64_t N, int sms) {
