@@ -174,3 +174,21 @@ def test_neox_decode_layer_sampled(zq, monkeypatch):
     a_split = zq.zq_w8a8_linear(*args, out_kind=zq.ZQ_OUT_I32_RAW)
     assert torch.equal(a_model, a_split)
     np.testing.assert_array_equal(host(a_model)[:, cols], acc)
+
+
+def test_largest_k_closed_form(zq, monkeypatch):
+    """All codes +-127 at the largest legal K (a multiple of 16, its last
+    k-block 16 bytes) through the even split: one weight tile's 1041 k-blocks
+    spread over the SMs (about 8 a CTA, so about 130 partial sums per
+    output), acc = +-127^2 K exactly, and the same with a ragged second tile
+    (N = 144)."""
+    monkeypatch.setenv("ZQ_EVEN_SPLIT", "on")
+    K = zq.ZQ_MAX_K // 16 * 16
+    for T, N in [(16, 128), (64, 144)]:
+        xq = torch.full((T, K), 127, dtype=torch.int8, device="cuda")
+        Wq = torch.full((N, K), 127, dtype=torch.int8, device="cuda")
+        Wq[1::2] = -127
+        acc = host(zq.zq_w8a8_linear(xq, torch.ones(T, device="cuda"), Wq, torch.ones(N, device="cuda"), 16,
+                                     out_kind=zq.ZQ_OUT_I32_RAW))
+        expect = np.where(np.arange(N) % 2 == 0, 127 * 127 * K, -127 * 127 * K)
+        np.testing.assert_array_equal(acc, np.broadcast_to(expect, (T, N)))
