@@ -925,7 +925,7 @@ def main(argv=None):
     peaks = load_peaks()
     dom = dominant_stage(stage_ms, stage_launches)
     roof = dict(stage_roofline(W, dom, stage_ms[dom], peaks, a.workload),
-                kernel=dom if dom.endswith("quant") else f"w8a8 linear ({dom})",
+                kernel=f"w8a8 linear ({dom})" if dom.startswith("linear") else dom,
                 launches_in_stage=stage_launches.get(dom))
     qlabel = "ln_quant" if "ln_quant" in stage_ms else ("act_quant" if "act_quant" in stage_ms else None)
     qb = W.kernel_units[qlabel][1] if qlabel else 0
