@@ -96,9 +96,24 @@ def _lin(**kw):
     (dict(out=zq.ZQ_OUT_I32_RAW, bias=A16), zq.ZQ_ERR_DTYPE),
     (dict(out=zq.ZQ_OUT_I8_REQUANT, s_out=A16b, ws=None, ws_bytes=0), zq.ZQ_ERR_WORKSPACE),
     (dict(out=zq.ZQ_OUT_I8_REQUANT, s_out=A16b, ws=A16c, ws_bytes=100), zq.ZQ_ERR_WORKSPACE),
+    # the optional workspace of the other kinds, when given, is 16-byte aligned
+    (dict(T=16, out=zq.ZQ_OUT_BF16, ws=MIS, ws_bytes=1 << 20), zq.ZQ_ERR_ALIGN),
+    (dict(T=16, out=zq.ZQ_OUT_I32_RAW, ws=A16c + 8, ws_bytes=1 << 20), zq.ZQ_ERR_ALIGN),
 ])
 def test_linear_rejects_bad_arguments_on_host(kw, status):
     assert _lin(**kw) == status
+
+
+def test_optional_workspace_without_a_device():
+    """The few-token even split needs the SM count; with no usable device the
+    query offers no workspace for the non-requantizing kinds (a call then
+    takes the split-K clusters), whatever the shape."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    for T, K, N in [(16, 6144, 24576), (1, 128, 16), (64, 4096, 65536), (65, 6144, 24576)]:
+        for kind in (zq.ZQ_OUT_F32, zq.ZQ_OUT_BF16, zq.ZQ_OUT_I32_RAW):
+            assert zq.lib().zq_w8a8_linear_workspace(T, K, N, kind) == 0
 
 
 def test_max_k_is_the_int32_bound():
